@@ -1,0 +1,155 @@
+"""TEST INFRASTRUCTURE — Python front end of the fp64 MLA decode oracle.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg
+use this module.  It never imports the CUDA package: callers hand it arrays
+(bf16 passed as uint16 bit patterns).
+
+Two independent fp64 implementations of the same definition live here:
+
+* ``mla_decode`` / ``mla_decode_etap`` — the C oracle (``mla_oracle.c``), in the
+  standard form S = Q K^T, P = softmax(S), O = P V and in the transposed ETAP
+  form S^T = K Q^T, P^T = softmax(S^T), O^T = V^T P^T, O = (O^T)^T
+  (FlashMLA-ETAP technical summary, "Methodology", the ETAP step list);
+* ``mla_decode_numpy`` — the standard form written with numpy fp64 matmuls, used
+  to cross-check the C code.
+
+``lse_merge`` is the log-sum-exp merge of results over disjoint KV ranges.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+D_QK = 576
+D_V = 512
+PAGE = 64
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mla_oracle.c")
+_LIB = os.path.join(_HERE, "libmla_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle (gcc, OpenMP) next to its source; returns the .so path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        args = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                ctypes.c_void_p, ctypes.c_void_p]
+        for name in ("oracle_mla_decode", "oracle_mla_decode_etap"):
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int
+        lib.oracle_lse_merge.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p]
+        lib.oracle_lse_merge.restype = None
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _call(name, q_bits, kv_bits, seqlens, block_table, scale, causal, threads=None):
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    kv_bits = np.ascontiguousarray(kv_bits, dtype=np.uint16)
+    seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
+    B, q_len, h, dqk = q_bits.shape
+    assert dqk == D_QK and kv_bits.shape[-1] == D_QK
+    if block_table is not None:
+        block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+        kv_rows, max_blocks, page = 0, block_table.shape[1], kv_bits.shape[1]
+    else:
+        kv_rows, max_blocks, page = kv_bits.shape[1], 0, PAGE
+    o = np.zeros((B, q_len, h, D_V), dtype=np.float64)
+    lse = np.zeros((B, q_len, h), dtype=np.float64)
+    if threads is not None:
+        os.environ["OMP_NUM_THREADS"] = str(threads)
+    rc = getattr(_load(), name)(_ptr(q_bits), _ptr(kv_bits), _ptr(seqlens), _ptr(block_table),
+                                B, q_len, h, D_QK, D_V, kv_rows, max_blocks, page,
+                                float(scale), int(bool(causal)), _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise MemoryError(f"{name} failed ({rc})")
+    return o, lse
+
+
+def mla_decode(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.0, causal=False):
+    """Standard-form oracle.  Returns (O fp64 [B,q,h,512], LSE fp64 [B,q,h])."""
+    return _call("oracle_mla_decode", q_bits, kv_bits, seqlens, block_table, scale, causal)
+
+
+def mla_decode_etap(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.0, causal=False):
+    """Transposed-form (ETAP steps 1-4) oracle.  Same outputs as ``mla_decode``."""
+    return _call("oracle_mla_decode_etap", q_bits, kv_bits, seqlens, block_table, scale, causal)
+
+
+def lse_merge(o_s: np.ndarray, lse_s: np.ndarray):
+    """Merge S partial results over disjoint KV ranges: o_s [S, d], lse_s [S] -> (o [d], lse)."""
+    o_s = np.ascontiguousarray(o_s, dtype=np.float64)
+    lse_s = np.ascontiguousarray(lse_s, dtype=np.float64)
+    S, d = o_s.shape
+    o = np.zeros(d, dtype=np.float64)
+    lse = np.zeros(1, dtype=np.float64)
+    _load().oracle_lse_merge(S, d, _ptr(o_s), _ptr(lse_s), _ptr(o), _ptr(lse))
+    return o, float(lse[0])
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to fp64."""
+    u = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
+def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to bf16 (nearest-even via fp32), returning bit patterns; for building test inputs."""
+    f = np.ascontiguousarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def mla_decode_numpy(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.0, causal=False):
+    """Second, independent fp64 implementation of the standard form with numpy matmuls."""
+    q = bf16_bits_to_f64(q_bits)
+    kv = bf16_bits_to_f64(kv_bits)
+    B, q_len, h, _ = q.shape
+    o = np.zeros((B, q_len, h, D_V))
+    lse = np.zeros((B, q_len, h))
+    for b in range(B):
+        L = int(seqlens[b])
+        if block_table is not None:
+            page = kv.shape[1]
+            nb = (L + page - 1) // page
+            rows = kv[np.asarray(block_table[b, :nb], dtype=np.int64)].reshape(nb * page, D_QK)[:L]
+        else:
+            rows = kv[b, :L]
+        for t in range(q_len):
+            vis = max(L - q_len + t + 1, 0) if causal else L
+            if vis == 0:
+                lse[b, t] = -math.inf
+                continue
+            S = scale * (q[b, t] @ rows[:vis].T)          # [h, vis]
+            m = S.max(axis=1, keepdims=True)
+            E = np.exp(S - m)
+            den = E.sum(axis=1, keepdims=True)
+            o[b, t] = (E / den) @ rows[:vis, :D_V]
+            lse[b, t] = (m + np.log(den))[:, 0]
+    return o, lse
