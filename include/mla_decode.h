@@ -1,0 +1,158 @@
+/*
+ * mla_decode.h — C ABI of libmla_decode.so: Multi-Head Latent Attention decode
+ * in the Efficient Transpose Attention Pipeline (ETAP) form, for NVIDIA B200 (sm_100a).
+ *
+ * Operation (FlashMLA-ETAP technical summary, "Methodology"): for every sequence
+ * b, query token t and head hd, with the N = q_len*h query columns ordered
+ * n = t*h + hd,
+ *     S^T = K Q^T          (KV rows are the MMA M dimension, query columns are N)
+ *     P^T = softmax(S^T)   over the KV rows of each column, after multiplying by softmax_scale
+ *     O^T = V^T P^T,  O = (O^T)^T
+ * K is the full 576-column latent row and V its first 512 columns (one shared
+ * latent KV head, the pages' "low-rank joint compression"). LSE is the natural
+ * log of the softmax denominator, scale included: LSE = ln sum_j exp(scale*q.k_j).
+ *
+ * Visible rows: j < L_b; with `causal` set, query token t sees rows
+ * j <= L_b - q_len + t (the q_len new tokens are the last q_len cache rows).
+ * A column with no visible row yields O = 0 and LSE = -inf.
+ *
+ * Conventions shared by every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; no call
+ *    allocates or frees memory and no call synchronises the host, except
+ *    mla_decode_read_status which waits for its own copy.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream).
+ *  - Arguments are validated on the host before anything is launched; an
+ *    invalid call returns an error code and launches nothing.
+ *  - Device-side problems (a wait that ran out of time, an out-of-range block
+ *    table entry) are recorded in a status word inside the workspace; read it
+ *    with mla_decode_read_status.
+ *  - Layouts are row-major; bf16 tensors are passed as void*.
+ */
+#ifndef MLA_DECODE_H
+#define MLA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mla_status {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = -1,   /* null pointer, bad size, bad scale, inconsistent arguments */
+    MLA_ERR_UNSUPPORTED = -2,   /* a shape this library does not implement */
+    MLA_ERR_ALIGNMENT = -3,     /* a pointer misses its required alignment */
+    MLA_ERR_WORKSPACE = -4,     /* workspace too small for (batch, q_len, num_heads, num_sms) */
+    MLA_ERR_CUDA = -5,          /* a CUDA runtime/driver call failed (see mla_last_cuda_error) */
+    MLA_ERR_TIMEOUT = -6,       /* device status: a bounded wait inside a kernel ran out */
+    MLA_ERR_BLOCK_TABLE = -7    /* device status: a block-table entry was outside [0, kv_rows) */
+} mla_status;
+
+enum {
+    MLA_D_QK = 576,      /* latent row width: 512 "nope" (also V) + 64 rope columns */
+    MLA_D_V = 512,       /* value width: the first 512 latent columns */
+    MLA_PAGE_SIZE = 64,  /* tokens per page of a paged cache */
+    MLA_MAX_BATCH = 65536,
+    MLA_MAX_COLUMNS = 1024 /* max q_len * num_heads */
+};
+
+/* Flags for mla_decode_fwd. */
+enum {
+    MLA_FLAG_SKIP_COMBINE = 1 /* leave split partials in the workspace; call mla_combine yourself */
+};
+
+/*
+ * Bytes of device workspace the plan/fwd/combine calls need for this shape.
+ * num_sms is the number of SMs to spread the work over (148 on a B200).
+ * Returns 0 for invalid arguments.
+ *
+ * Workspace layout (owned by the caller, 256-byte aligned): a small header
+ * (status word, plan sizes), the split-KV schedule written by mla_decode_plan,
+ * then fp32 partial outputs [slots, q_len*h, 512] and partial LSEs for
+ * sequences whose KV range is split over several CTAs.
+ */
+MLA_API size_t mla_decode_workspace_size(int batch, int q_len, int num_heads, int num_sms);
+
+/*
+ * Split-KV scheduling metadata (not on the pages: needed so that a batch with
+ * few sequences still fills every SM). Reads seqlens (device int32[batch]),
+ * cuts the concatenated KV tiles (128 rows each) of all sequences into
+ * num_ctas near-equal contiguous ranges, and records for each sequence how
+ * many ranges touch it and where its partial results go. One small kernel;
+ * no host synchronisation, so the call can be captured in a CUDA graph.
+ * Also clears the workspace status word.
+ */
+MLA_API int mla_decode_plan(const int32_t *seqlens, int batch, int q_len, int num_heads, int num_sms,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The decode itself (ETAP steps 1-4 of the pages, plus the split-KV partial
+ * outputs and, unless MLA_FLAG_SKIP_COMBINE is set, the combine).
+ *   q            bf16 [batch, q_len, num_heads, 576], 16-byte aligned
+ *   kv           contiguous: bf16 [batch, kv_rows, 576];
+ *                paged (block_table != NULL): bf16 [kv_rows / 64, 64, 576], i.e. kv_rows = num_blocks*64
+ *   seqlens      int32 [batch], device, 0 <= L_b (<= kv_rows when contiguous;
+ *                <= max_blocks*64 when paged)
+ *   block_table  int32 [batch, max_blocks] of physical block ids, or NULL for a contiguous cache.
+ *                Entries past ceil(L_b/64) are never read. An entry outside
+ *                [0, kv_rows/64) is not dereferenced: that page is not loaded, the
+ *                sequence's output is unspecified, and MLA_ERR_BLOCK_TABLE is set in
+ *                the status word.
+ *   softmax_scale  > 0 and finite (576^-0.5 for the DeepSeek-R1 shape)
+ *   causal       0 or 1 (see the header comment)
+ *   o            bf16 [batch, q_len, num_heads, 512], 16-byte aligned
+ *   lse          fp32 [batch, q_len, num_heads], 4-byte aligned
+ *   workspace    the buffer mla_decode_plan filled for the same seqlens and shape
+ * Rows of the cache past L_b may hold anything (NaN included): they are masked
+ * out and never multiply into O.
+ */
+MLA_API int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const int32_t *block_table,
+                   int batch, int q_len, int num_heads, int64_t kv_rows, int max_blocks,
+                   float softmax_scale, int causal, void *o, float *lse,
+                   void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream);
+
+/*
+ * Log-sum-exp merge of the split-KV partials that mla_decode_fwd left in the
+ * workspace: lse = ln sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s, for
+ * every sequence split over several CTAs; also writes O = 0, LSE = -inf for
+ * empty sequences. Sequences handled by one CTA were already written by fwd.
+ */
+MLA_API int mla_combine(const void *workspace, int batch, int q_len, int num_heads, int num_sms,
+                void *o, float *lse, void *stream);
+
+/*
+ * Copy the workspace status word to the host (waits for that copy only).
+ * *status_out receives MLA_OK or the first device-side error recorded.
+ */
+MLA_API int mla_decode_read_status(const void *workspace, int *status_out, void *stream);
+
+/*
+ * Host mirror of the split-KV schedule, for testing and for callers that
+ * want to inspect it. seqlens is a HOST int32[batch]. Writes, when the
+ * pointers are non-NULL:
+ *   cta_ranges  int32[num_ctas*2]  flattened tile range [begin, end) of each CTA
+ *   seq_info    int32[batch*4]     per sequence: tile count, first CTA, number of splits, partial slot offset
+ * and returns the number of CTAs per column group (num_ctas) through *num_ctas_out.
+ */
+MLA_API int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, int num_heads, int num_sms,
+                         int32_t *cta_ranges, int32_t *seq_info, int *num_ctas_out, int *num_groups_out);
+
+/* Human-readable name of a status code. */
+MLA_API const char *mla_status_string(int status);
+
+/* The last CUDA error string seen by this thread (after MLA_ERR_CUDA). */
+MLA_API const char *mla_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H */

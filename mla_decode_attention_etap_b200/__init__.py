@@ -1,0 +1,179 @@
+"""Python binding of libmla_decode.so: MLA decode attention in the ETAP form on B200.
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels.  torch tensors provide device memory and the current stream.
+The names mirror the C ABI in ``include/mla_decode.h``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla_decode.so")
+
+D_QK = 576
+D_V = 512
+PAGE_SIZE = 64
+FLAG_SKIP_COMBINE = 1
+
+STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3: "MLA_ERR_ALIGNMENT",
+          -4: "MLA_ERR_WORKSPACE", -5: "MLA_ERR_CUDA", -6: "MLA_ERR_TIMEOUT", -7: "MLA_ERR_BLOCK_TABLE"}
+
+EXPORTS = ("mla_decode_workspace_size", "mla_decode_plan", "mla_decode_fwd", "mla_combine",
+           "mla_decode_read_status", "mla_decode_plan_host", "mla_status_string", "mla_last_cuda_error")
+
+
+class MlaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library.  Raises if it was not built (no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m mla_decode_attention_etap_b200.build` "
+                              "(or __graft_entry__.build()) first; there is no non-CUDA fallback")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        L.mla_decode_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.mla_decode_workspace_size.restype = sz
+        L.mla_decode_plan.argtypes = [vp, i32, i32, i32, i32, vp, sz, vp]
+        L.mla_decode_plan.restype = i32
+        L.mla_decode_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp, vp, vp, sz,
+                                     i32, ctypes.c_uint, vp]
+        L.mla_decode_fwd.restype = i32
+        L.mla_combine.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
+        L.mla_combine.restype = i32
+        L.mla_decode_read_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
+        L.mla_decode_read_status.restype = i32
+        L.mla_decode_plan_host.argtypes = [vp, i32, i32, i32, i32, vp, vp, ctypes.POINTER(ctypes.c_int),
+                                           ctypes.POINTER(ctypes.c_int)]
+        L.mla_decode_plan_host.restype = i32
+        L.mla_status_string.argtypes = [i32]
+        L.mla_status_string.restype = ctypes.c_char_p
+        L.mla_last_cuda_error.argtypes = []
+        L.mla_last_cuda_error.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        if code == -5:
+            what = f"{what} ({lib().mla_last_cuda_error().decode()})"
+        raise MlaError(code, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def num_sms(device=None) -> int:
+    return torch.cuda.get_device_properties(device if device is not None else torch.cuda.current_device()
+                                            ).multi_processor_count
+
+
+def mla_decode_workspace_size(batch: int, q_len: int, num_heads: int, n_sms: int) -> int:
+    n = lib().mla_decode_workspace_size(batch, q_len, num_heads, n_sms)
+    if n == 0:
+        raise MlaError(-1, "mla_decode_workspace_size")
+    return int(n)
+
+
+def mla_decode_plan(seqlens: torch.Tensor, q_len: int, num_heads: int, workspace: torch.Tensor, n_sms: int,
+                    stream=None) -> None:
+    _check(lib().mla_decode_plan(_ptr(seqlens), seqlens.numel(), q_len, num_heads, n_sms, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)), "mla_decode_plan")
+
+
+def mla_decode_fwd(q, kv, seqlens, block_table, softmax_scale, causal, o, lse, workspace, n_sms, flags=0,
+                   stream=None) -> None:
+    B, q_len, h, _ = q.shape
+    if block_table is not None:
+        kv_rows, max_blocks = kv.shape[0] * kv.shape[1], block_table.shape[1]
+    else:
+        kv_rows, max_blocks = kv.shape[1], 0
+    _check(lib().mla_decode_fwd(_ptr(q), _ptr(kv), _ptr(seqlens), _ptr(block_table), B, q_len, h, kv_rows,
+                                max_blocks, float(softmax_scale), int(bool(causal)), _ptr(o), _ptr(lse),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(), n_sms, flags,
+                                _stream(stream)), "mla_decode_fwd")
+
+
+def mla_combine(workspace, batch, q_len, num_heads, n_sms, o, lse, stream=None) -> None:
+    _check(lib().mla_combine(_ptr(workspace), batch, q_len, num_heads, n_sms, _ptr(o), _ptr(lse), _stream(stream)),
+           "mla_combine")
+
+
+def mla_decode_read_status(workspace, stream=None) -> int:
+    out = ctypes.c_int(0)
+    _check(lib().mla_decode_read_status(_ptr(workspace), ctypes.byref(out), _stream(stream)),
+           "mla_decode_read_status")
+    return int(out.value)
+
+
+def mla_decode_plan_host(seqlens, q_len: int, num_heads: int, n_sms: int):
+    """Host mirror of the schedule -> (cta_ranges [ctas, 2], seq_info [B, 4], num_ctas, num_groups)."""
+    import numpy as np
+    sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    nct, ngr = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().mla_decode_plan_host(sl.ctypes.data_as(ctypes.c_void_p), sl.size, q_len, num_heads, n_sms, None,
+                                      None, ctypes.byref(nct), ctypes.byref(ngr)), "mla_decode_plan_host")
+    ranges = np.zeros((nct.value, 2), np.int32)
+    info = np.zeros((sl.size, 4), np.int32)
+    _check(lib().mla_decode_plan_host(sl.ctypes.data_as(ctypes.c_void_p), sl.size, q_len, num_heads, n_sms,
+                                      ranges.ctypes.data_as(ctypes.c_void_p), info.ctypes.data_as(ctypes.c_void_p),
+                                      ctypes.byref(nct), ctypes.byref(ngr)), "mla_decode_plan_host")
+    return ranges, info, nct.value, ngr.value
+
+
+class MlaDecoder:
+    """Owns the workspace for one (batch, q_len, num_heads) shape; plan() then fwd()."""
+
+    def __init__(self, batch: int, q_len: int, num_heads: int, device=None, n_sms: Optional[int] = None):
+        self.device = torch.device(device if device is not None else "cuda")
+        self.batch, self.q_len, self.num_heads = batch, q_len, num_heads
+        self.n_sms = n_sms if n_sms is not None else num_sms(self.device)
+        nbytes = mla_decode_workspace_size(batch, q_len, num_heads, self.n_sms)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+
+    def plan(self, seqlens: torch.Tensor, stream=None):
+        mla_decode_plan(seqlens, self.q_len, self.num_heads, self.workspace, self.n_sms, stream)
+
+    def fwd(self, q, kv, seqlens, block_table=None, softmax_scale=None, causal=False, o=None, lse=None,
+            flags=0, stream=None):
+        B, q_len, h, _ = q.shape
+        if o is None:
+            o = torch.empty(B, q_len, h, D_V, dtype=torch.bfloat16, device=q.device)
+        if lse is None:
+            lse = torch.empty(B, q_len, h, dtype=torch.float32, device=q.device)
+        scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(D_QK)
+        mla_decode_fwd(q, kv, seqlens, block_table, scale, causal, o, lse, self.workspace, self.n_sms, flags,
+                       stream)
+        return o, lse
+
+    def status(self, stream=None) -> int:
+        return mla_decode_read_status(self.workspace, stream)
+
+
+def mla_decode(q, kv, seqlens, block_table=None, softmax_scale=None, causal=False):
+    """One-shot convenience: plan + decode (+ combine).  Returns (O bf16, LSE fp32)."""
+    dec = MlaDecoder(q.shape[0], q.shape[1], q.shape[2], device=q.device)
+    dec.plan(seqlens)
+    return dec.fwd(q, kv, seqlens, block_table, softmax_scale, causal)

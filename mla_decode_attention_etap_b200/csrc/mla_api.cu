@@ -1,0 +1,272 @@
+// C ABI of libmla_decode.so (declared in include/mla_decode.h): argument
+// validation, TMA tensor-map encoding and the three launches (plan, ETAP
+// decode, combine).  No call allocates device memory or synchronises the host
+// (except mla_decode_read_status, which waits for its own 4-byte copy).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/mla_decode.h"
+#include "etap_decode_kernel.cuh"
+#include "plan_combine_kernels.cuh"
+#include "plan_core.h"
+
+namespace {
+
+thread_local std::string g_last_cuda_error;
+
+int cuda_fail(cudaError_t e, const char *what) {
+    g_last_cuda_error = std::string(what) + ": " + cudaGetErrorString(e);
+    return MLA_ERR_CUDA;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor map over a [rows, 576] row-major matrix; box = 64 columns x box_rows rows, 128B swizzle.
+int encode_rows_576(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) {
+        g_last_cuda_error = "cuTensorMapEncodeTiled unavailable";
+        return MLA_ERR_CUDA;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)mla::kDqk, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)mla::kDqk * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string((int)r);
+        return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+
+int check_shape(int batch, int q_len, int num_heads, int num_sms) {
+    if (batch < 1 || batch > MLA_MAX_BATCH) return MLA_ERR_INVALID_ARG;
+    if (q_len < 1 || num_heads < 1) return MLA_ERR_INVALID_ARG;
+    if ((int64_t)q_len * num_heads > MLA_MAX_COLUMNS) return MLA_ERR_UNSUPPORTED;
+    if (num_sms < 1 || num_sms > 4096) return MLA_ERR_INVALID_ARG;
+    return MLA_OK;
+}
+
+// Per-device one-time opt-in to the kernel's dynamic shared memory size.
+int ensure_smem_attr() {
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return MLA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+        e = cudaFuncSetAttribute(mla::etap_decode_kernel<mla::Cfg16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)mla::Cfg16::SMEM_ALLOC);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        done[dev] = true;
+    }
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mla_status_string(int status) {
+    switch (status) {
+        case MLA_OK: return "MLA_OK";
+        case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+        case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+        case MLA_ERR_ALIGNMENT: return "MLA_ERR_ALIGNMENT";
+        case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE";
+        case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+        case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT";
+        case MLA_ERR_BLOCK_TABLE: return "MLA_ERR_BLOCK_TABLE";
+        default: return "MLA_ERR_UNKNOWN";
+    }
+}
+
+const char *mla_last_cuda_error(void) { return g_last_cuda_error.c_str(); }
+
+size_t mla_decode_workspace_size(int batch, int q_len, int num_heads, int num_sms) {
+    if (check_shape(batch, q_len, num_heads, num_sms) != MLA_OK) return 0;
+    return mla::ws_layout(batch, q_len, num_heads, num_sms).total;
+}
+
+int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, int num_heads, int num_sms,
+                         int32_t *cta_ranges, int32_t *seq_info, int *num_ctas_out, int *num_groups_out) {
+    int st = check_shape(batch, q_len, num_heads, num_sms);
+    if (st != MLA_OK) return st;
+    if (!seqlens) return MLA_ERR_INVALID_ARG;
+    const mla::WsLayout lay = mla::ws_layout(batch, q_len, num_heads, num_sms);
+    int64_t total = 0;
+    for (int b = 0; b < batch; ++b) total += mla::tiles_of(seqlens[b]);
+    if (total > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+    const int used = mla::used_ctas(total, lay.ctas);
+    if (cta_ranges)
+        for (int c = 0; c < lay.ctas; ++c) {
+            cta_ranges[2 * c] = (int32_t)mla::cta_begin(total, used, c);
+            cta_ranges[2 * c + 1] = (int32_t)mla::cta_begin(total, used, c + 1);
+        }
+    if (seq_info) {
+        int64_t off = 0;
+        int slots = 0;
+        for (int b = 0; b < batch; ++b) {
+            const int64_t t0 = off, t1 = off + mla::tiles_of(seqlens[b]);
+            int first = -1, nsplit = 0;
+            if (t1 > t0) {
+                first = mla::cta_of(total, used, t0);
+                nsplit = mla::cta_of(total, used, t1 - 1) - first + 1;
+            }
+            seq_info[4 * b + 0] = (int32_t)(t1 - t0);
+            seq_info[4 * b + 1] = first;
+            seq_info[4 * b + 2] = nsplit;
+            seq_info[4 * b + 3] = slots;
+            if (nsplit >= 2) slots += nsplit;
+            off = t1;
+        }
+    }
+    if (num_ctas_out) *num_ctas_out = lay.ctas;
+    if (num_groups_out) *num_groups_out = lay.groups;
+    return MLA_OK;
+}
+
+int mla_decode_plan(const int32_t *seqlens, int batch, int q_len, int num_heads, int num_sms, void *workspace,
+                    size_t workspace_bytes, void *stream) {
+    int st = check_shape(batch, q_len, num_heads, num_sms);
+    if (st != MLA_OK) return st;
+    if (!seqlens || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!aligned(seqlens, 4) || !aligned(workspace, 256)) return MLA_ERR_ALIGNMENT;
+    const mla::WsLayout lay = mla::ws_layout(batch, q_len, num_heads, num_sms);
+    if (workspace_bytes < lay.total) return MLA_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    mla::plan_kernel<<<1, 256, 0, s>>>(seqlens, batch, lay.ctas, lay.groups, q_len * num_heads,
+                                       reinterpret_cast<int32_t *>(workspace), lay);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "plan_kernel launch");
+    return MLA_OK;
+}
+
+int mla_combine(const void *workspace, int batch, int q_len, int num_heads, int num_sms, void *o, float *lse,
+                void *stream) {
+    int st = check_shape(batch, q_len, num_heads, num_sms);
+    if (st != MLA_OK) return st;
+    if (!workspace || !o || !lse) return MLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256) || !aligned(o, 16) || !aligned(lse, 4)) return MLA_ERR_ALIGNMENT;
+    const mla::WsLayout lay = mla::ws_layout(batch, q_len, num_heads, num_sms);
+    const int ncols = q_len * num_heads;
+    const char *ws = reinterpret_cast<const char *>(workspace);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    mla::combine_kernel<<<dim3(ncols, batch), 128, 0, s>>>(
+        reinterpret_cast<const int32_t *>(ws), reinterpret_cast<const float *>(ws + lay.opart),
+        reinterpret_cast<const float *>(ws + lay.lsepart), ncols, lay, reinterpret_cast<__nv_bfloat16 *>(o), lse);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "combine_kernel launch");
+    return MLA_OK;
+}
+
+int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const int32_t *block_table, int batch,
+                   int q_len, int num_heads, int64_t kv_rows, int max_blocks, float softmax_scale, int causal,
+                   void *o, float *lse, void *workspace, size_t workspace_bytes, int num_sms, unsigned flags,
+                   void *stream) {
+    int st = check_shape(batch, q_len, num_heads, num_sms);
+    if (st != MLA_OK) return st;
+    if (!q || !kv || !seqlens || !o || !lse || !workspace) return MLA_ERR_INVALID_ARG;
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
+    if ((flags & ~(unsigned)MLA_FLAG_SKIP_COMBINE) != 0) return MLA_ERR_INVALID_ARG;
+    if (kv_rows < 1) return MLA_ERR_INVALID_ARG;
+    const bool paged = block_table != nullptr;
+    if (paged) {
+        if (kv_rows % MLA_PAGE_SIZE != 0 || max_blocks < 1) return MLA_ERR_INVALID_ARG;
+        if (kv_rows > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+        if (!aligned(block_table, 4)) return MLA_ERR_ALIGNMENT;
+    } else {
+        if ((int64_t)batch * kv_rows > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+    }
+    if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(o, 16) || !aligned(lse, 4) || !aligned(seqlens, 4) ||
+        !aligned(workspace, 256))
+        return MLA_ERR_ALIGNMENT;
+    const mla::WsLayout lay = mla::ws_layout(batch, q_len, num_heads, num_sms);
+    if (workspace_bytes < lay.total) return MLA_ERR_WORKSPACE;
+    const int ncols = q_len * num_heads;
+
+    st = ensure_smem_attr();
+    if (st != MLA_OK) return st;
+    CUtensorMap tm_q, tm_kv;
+    st = encode_rows_576(&tm_q, q, (uint64_t)batch * ncols, mla::Cfg16::NG);
+    if (st != MLA_OK) return st;
+    st = encode_rows_576(&tm_kv, kv, paged ? (uint64_t)kv_rows : (uint64_t)batch * kv_rows, 64);
+    if (st != MLA_OK) return st;
+
+    char *ws = reinterpret_cast<char *>(workspace);
+    mla::DecodeParams p{};
+    p.seqlens = seqlens;
+    p.block_table = block_table;
+    p.ws = reinterpret_cast<int32_t *>(ws);
+    p.opart = reinterpret_cast<float *>(ws + lay.opart);
+    p.lsepart = reinterpret_cast<float *>(ws + lay.lsepart);
+    p.o = reinterpret_cast<__nv_bfloat16 *>(o);
+    p.lse = lse;
+    p.kv_rows = kv_rows;
+    p.batch = batch;
+    p.q_len = q_len;
+    p.num_heads = num_heads;
+    p.ncols = ncols;
+    p.ctas = lay.ctas;
+    p.groups = lay.groups;
+    p.max_blocks = paged ? max_blocks : 0;
+    p.paged = paged ? 1 : 0;
+    p.causal = causal;
+    p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.cta_ranges_off = (int)(lay.cta_ranges / 4);
+    p.tile_off_off = (int)(lay.tile_off / 4);
+    p.seq_info_off = (int)(lay.seq_info / 4);
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    mla::etap_decode_kernel<mla::Cfg16><<<lay.ctas * lay.groups, 192, mla::Cfg16::SMEM_ALLOC, s>>>(tm_q, tm_kv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "etap_decode_kernel launch");
+    if (!(flags & MLA_FLAG_SKIP_COMBINE))
+        return mla_combine(workspace, batch, q_len, num_heads, num_sms, o, lse, stream);
+    return MLA_OK;
+}
+
+int mla_decode_read_status(const void *workspace, int *status_out, void *stream) {
+    if (!workspace || !status_out) return MLA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return MLA_ERR_ALIGNMENT;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e, "status copy");
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "status copy sync");
+    *status_out = v;
+    return MLA_OK;
+}
+
+}  // extern "C"

@@ -62,7 +62,7 @@ class Workload:
             out = self.kv[b, :L]
         else:
             nb = (L + PAGE - 1) // PAGE
-            blocks = self.block_table[b, :nb].long()
+            blocks = self.block_table[b, :nb].long().to(self.kv.device)
             out = self.kv[blocks].reshape(nb * PAGE, D_QK)[:L]
         return out if rows is None else out[rows]
 

@@ -1,0 +1,83 @@
+"""Shared helpers for the parity tests: run the CUDA path and the oracle on the same inputs."""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from mla_decode_attention_etap_b200 import MlaDecoder
+from mla_decode_attention_etap_b200.workloads import Workload, bf16_bits
+from oracle import mla_oracle as om
+
+# Tolerances of the parity bar, applied to the whole compared tensor:
+RMSE_REL = 2e-3     # RMSE(O - O_ref) <= 2e-3 * RMS(O_ref)
+MAXABS_REL = 1e-2   # max|O - O_ref| <= 1e-2 * max|O_ref|
+LSE_ABS = 1e-3      # max|LSE - LSE_ref| <= 1e-3 (natural log)
+
+
+def run_cuda(w: Workload, n_sms=None, flags=0, poison=True, decoder=None):
+    """Plan + decode (+ combine) through the C ABI; outputs pre-filled with NaN to catch holes."""
+    dev = torch.device("cuda")
+    q = w.q.to(dev)
+    kv = w.kv.to(dev)
+    sl = w.seqlens.to(dev)
+    bt = w.block_table.to(dev) if w.block_table is not None else None
+    dec = decoder or MlaDecoder(w.batch, w.q_len, w.num_heads, device=dev, n_sms=n_sms)
+    o = torch.full((w.batch, w.q_len, w.num_heads, 512), float("nan") if poison else 0.0,
+                   dtype=torch.bfloat16, device=dev)
+    lse = torch.full((w.batch, w.q_len, w.num_heads), float("nan") if poison else 0.0,
+                     dtype=torch.float32, device=dev)
+    dec.plan(sl)
+    dec.fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o=o, lse=lse, flags=flags)
+    torch.cuda.synchronize()
+    status = dec.status()
+    return o.float().cpu().numpy(), lse.cpu().numpy(), status, dec
+
+
+def run_oracle(w: Workload, batch_index=None):
+    """fp64 oracle on all sequences, or on the listed ones (each resolved to a contiguous copy)."""
+    if batch_index is None:
+        q = bf16_bits(w.q)
+        kv = bf16_bits(w.kv)
+        bt = None if w.block_table is None else w.block_table.numpy()
+        return om.mla_decode(q, kv, w.seqlens.numpy(), bt, w.softmax_scale, w.causal)
+    outs_o, outs_l = [], []
+    for b in batch_index:
+        L = int(w.seqlens[b])
+        rows = w.kv_rows(b).cpu()
+        kv = bf16_bits(rows.reshape(1, max(L, 0), 576)) if L > 0 else np.zeros((1, 1, 576), np.uint16)
+        q = bf16_bits(w.q[b:b + 1].cpu())
+        o, lse = om.mla_decode(q, kv, np.array([L], np.int32), None, w.softmax_scale, w.causal)
+        outs_o.append(o[0])
+        outs_l.append(lse[0])
+    return np.stack(outs_o), np.stack(outs_l)
+
+
+def parity_metrics(o, lse, o_ref, lse_ref):
+    o = np.asarray(o, np.float64)
+    o_ref = np.asarray(o_ref, np.float64)
+    err = o - o_ref
+    rms_ref = math.sqrt(float(np.mean(o_ref ** 2))) if o_ref.size else 0.0
+    rmse = math.sqrt(float(np.mean(err ** 2))) if err.size else 0.0
+    finite = np.isfinite(lse_ref)
+    lse_err = float(np.max(np.abs(lse[finite] - lse_ref[finite]))) if finite.any() else 0.0
+    return {
+        "rmse": rmse, "rms_ref": rms_ref, "rmse_rel": rmse / rms_ref if rms_ref > 0 else rmse,
+        "maxabs": float(np.max(np.abs(err))) if err.size else 0.0,
+        "max_ref": float(np.max(np.abs(o_ref))) if o_ref.size else 0.0,
+        "lse_err": lse_err,
+        "nan_o": int(np.isnan(o).sum()),
+        "inf_lse_mismatch": int(np.sum(np.isneginf(lse_ref) != np.isneginf(lse))),
+    }
+
+
+def assert_parity(o, lse, o_ref, lse_ref, what=""):
+    m = parity_metrics(o, lse, o_ref, lse_ref)
+    assert m["nan_o"] == 0, f"{what}: {m['nan_o']} NaN outputs {m}"
+    assert m["inf_lse_mismatch"] == 0, f"{what}: -inf LSE pattern differs {m}"
+    assert m["rmse"] <= RMSE_REL * m["rms_ref"] + 1e-12, f"{what}: RMSE {m}"
+    assert m["maxabs"] <= MAXABS_REL * m["max_ref"] + 1e-12, f"{what}: max-abs {m}"
+    assert m["lse_err"] <= LSE_ABS, f"{what}: LSE {m}"
+    return m

@@ -1,0 +1,193 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Small cases span several 128-row tiles and ragged tails and are compared in
+full; the full-size workloads run in the launch configuration of bench.py
+(148 SMs) and are compared on sampled sequences the oracle computes one by one.
+Tolerance (applied to each compared tensor): RMSE(O) <= 2e-3 RMS(O_ref),
+max|dO| <= 1e-2 max|O_ref|, max|dLSE| <= 1e-3.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from mla_decode_attention_etap_b200 import workloads as W
+from tests.parity import assert_parity, run_cuda, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _poison_padding(w: W.Workload):
+    """NaN in every cache row the sequences do not own: the kernel must never let it into O."""
+    nan = torch.tensor(float("nan"), dtype=torch.bfloat16)
+    if w.block_table is None:
+        for b in range(w.batch):
+            w.kv[b, int(w.seqlens[b]):] = nan
+    else:
+        used = set()
+        for b in range(w.batch):
+            L = int(w.seqlens[b])
+            nb = (L + 63) // 64
+            for i in range(nb):
+                blk = int(w.block_table[b, i])
+                used.add(blk)
+                if i == nb - 1 and L % 64:
+                    w.kv[blk, L % 64:] = nan
+        for blk in range(w.kv.shape[0]):
+            if blk not in used:
+                w.kv[blk] = nan
+    return w
+
+
+def test_b1_h16_l1024():
+    w = W.workload_b1_h16_l1024(seed=0)
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what="B=1 h=16 L=1024")
+
+
+@pytest.mark.parametrize("L", [1, 2, 63, 64, 65, 127, 128, 129, 511, 512, 513, 1000])
+def test_edge_lengths_single_sequence(L):
+    w = _poison_padding(W.make_workload(1, 16, [L], seed=L, l_max=L + 200))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"L={L}")
+
+
+def test_mixed_lengths_with_empty_sequence_and_nan_padding():
+    lens = [0, 1, 129, 700, 64, 2000, 3, 0]
+    w = _poison_padding(W.make_workload(len(lens), 16, lens, seed=3))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    o_ref, lse_ref = run_oracle(w)
+    assert np.all(o[0] == 0) and np.all(np.isneginf(lse[0]))
+    assert_parity(o, lse, o_ref, lse_ref, what="mixed")
+
+
+@pytest.mark.parametrize("n_sms", [1, 3, 16, 148, 300])
+def test_split_counts(n_sms):
+    """From one CTA walking every sequence to many CTAs per sequence (split + combine)."""
+    w = W.make_workload(3, 16, [3000, 257, 1536], seed=4)
+    o, lse, st, dec = run_cuda(w, n_sms=n_sms)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"n_sms={n_sms}")
+
+
+def test_paged_random_permutation_nan_elsewhere():
+    lens = [1, 64, 65, 300, 1234, 4096, 77]
+    w = _poison_padding(W.make_workload(len(lens), 16, lens, paged=True, seed=5, extra_blocks=7))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what="paged")
+
+
+@pytest.mark.parametrize("L", [2, 5, 100, 131, 700])
+def test_causal_q4(L):
+    w = W.make_workload(2, 16, [L, L + 37], q_len=4, causal=True, seed=6, spike_frac=0.05)
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"causal L={L}")
+
+
+def test_causal_shorter_than_q_len():
+    w = W.make_workload(1, 16, [2], q_len=4, causal=True, seed=7)
+    o, lse, st, _ = run_cuda(w)
+    o_ref, lse_ref = run_oracle(w)
+    assert np.all(np.isneginf(lse[0, :2])) and np.all(o[0, :2] == 0)
+    assert_parity(o, lse, o_ref, lse_ref, what="causal L<q")
+
+
+def test_h128_paged():
+    w = W.make_workload(3, 128, [300, 1100, 129], paged=True, seed=8)
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what="h=128")
+
+
+def test_odd_column_count():
+    """q_len*h not a multiple of 16: the last column group is partly empty."""
+    w = W.make_workload(2, 8, [500, 90], q_len=1, seed=9)
+    o, lse, st, _ = run_cuda(w)
+    assert_parity(o, lse, *run_oracle(w), what="h=8")
+    w = W.make_workload(2, 20, [333, 1], q_len=1, seed=10)
+    o, lse, st, _ = run_cuda(w)
+    assert_parity(o, lse, *run_oracle(w), what="h=20")
+
+
+def test_spiky_scores_force_rescale():
+    """Rows scaled x8 and x64 make running maxima jump (TMEM rescale path)."""
+    w = W.make_workload(2, 16, [5000, 3000], seed=11, spike_frac=0.05, spike_scale=8.0)
+    o, lse, st, _ = run_cuda(w)
+    assert_parity(o, lse, *run_oracle(w), what="spikes x8")
+    w = W.make_workload(1, 16, [4000], seed=12)
+    w.kv[0, 3500] = (w.kv[0, 3500].float() * 64).to(torch.bfloat16)
+    w.kv[0, 100] = (w.kv[0, 100].float() * 16).to(torch.bfloat16)
+    o, lse, st, _ = run_cuda(w)
+    assert_parity(o, lse, *run_oracle(w), what="spikes x64")
+
+
+def test_repeat_is_deterministic_and_skip_combine_path():
+    w = W.make_workload(2, 16, [4000, 900], seed=13)
+    o1, l1, _, dec = run_cuda(w)
+    o2, l2, _, _ = run_cuda(w, decoder=dec)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    # fwd without combine, then the separate combine call
+    from mla_decode_attention_etap_b200 import FLAG_SKIP_COMBINE, mla_combine
+    o3, l3, _, dec3 = run_cuda(w, flags=FLAG_SKIP_COMBINE, poison=False)
+    dev = torch.device("cuda")
+    o_t = torch.tensor(o3, dtype=torch.bfloat16, device=dev)
+    l_t = torch.tensor(l3, dtype=torch.float32, device=dev)
+    mla_combine(dec3.workspace, w.batch, w.q_len, w.num_heads, dec3.n_sms, o_t, l_t)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(o_t.float().cpu().numpy(), o1)
+    np.testing.assert_array_equal(l_t.cpu().numpy(), l1)
+
+
+def test_bad_block_table_entry_sets_status():
+    w = W.make_workload(2, 16, [200, 300], paged=True, seed=14)
+    w.block_table[1, 2] = 10 ** 6          # far outside the pool
+    w.block_table[0, 0] = -5
+    _, _, st, _ = run_cuda(w)
+    assert st == -7
+
+
+# ---------------------------------------------------------------- full-size workloads (sampled)
+def _full(w, sample):
+    o, lse, st, _ = run_cuda(w, poison=True)
+    assert st == 0
+    assert not np.isnan(o).any()
+    o_ref, lse_ref = run_oracle(w, sample)
+    return assert_parity(o[sample], lse[sample], o_ref, lse_ref, what="full-size sample")
+
+
+def test_full_b16_h16_64k_sampled():
+    w = W.workload_b16_h16(65536, seed=0, device="cuda")
+    _full(w, [0, 11])
+
+
+@pytest.mark.parametrize("L", [4096, 16384, 32768])
+def test_full_b16_h16_sweep_sampled(L):
+    w = W.workload_b16_h16(L, seed=0, device="cuda")
+    _full(w, [3])
+
+
+def test_full_b64_h16_paged_sampled():
+    w = W.workload_b64_h16_paged(seed=0, device="cuda")
+    lens = w.seqlens.tolist()
+    sample = [int(np.argmin(lens)), int(np.argmax(lens)), 17]
+    _full(w, sample)
+
+
+def test_full_b32_h128_paged_sampled():
+    w = W.workload_b32_h128_paged(seed=0, device="cuda")
+    _full(w, [5])
+
+
+def test_full_b16_h16_q4_causal_sampled():
+    w = W.workload_b16_h16_q4_causal(seed=0, device="cuda")
+    _full(w, [0, 9])
