@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Benchmark of MLA decode attention (ETAP form) on B200.
+
+One step = one pass of the whole decode path over one batch: split-KV plan,
+ETAP decode kernel, log-sum-exp combine.  Default workload: B=16 sequences,
+16 heads, one query token, 65536 contiguous cache rows each (1.21 GB of bf16
+latent KV, larger than the 126 MB L2, so no flush is needed between steps).
+
+Reported value: whole-job KV throughput in TB/s (algorithmic bytes: 1152 per
+cached token read once) over the max-over-ranks device time of K steps.  The
+line also carries TFLOPS (2*(576+512) flops per visible (query column, token)
+pair), the decode kernel's roofline fraction (live CUDA-event timing of that
+kernel on its stream), an end-to-end figure through the C ABI with host
+buffers, the fp64 oracle timed on the host as a CPU baseline, and GPU clocks
+sampled while the steps run.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank decodes its own
+batch (independent sequences, no collective on the data path: weak scaling).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode TB/s & TFLOPS (B=16,h=16,64K KV) as % of B200 roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+KERNEL_SOURCES = ["mla_decode_attention_etap_b200/csrc/etap_decode_kernel.cuh",
+                  "mla_decode_attention_etap_b200/csrc/ptx_sm100.cuh",
+                  "mla_decode_attention_etap_b200/csrc/plan_core.h"]
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "etap_decode_kernel_ncu.md")
+
+WORKLOADS = {
+    "b16_h16_64k": dict(batch=16, heads=16, seqlen=65536),
+    "b16_h16_32k": dict(batch=16, heads=16, seqlen=32768),
+    "b16_h16_16k": dict(batch=16, heads=16, seqlen=16384),
+    "b16_h16_4k": dict(batch=16, heads=16, seqlen=4096),
+    "b1_h16_1k": dict(batch=1, heads=16, seqlen=1024),
+    "b64_h16_paged": dict(kind="b64_paged"),
+    "b32_h128_paged": dict(kind="b32_h128"),
+    "b16_h16_q4_causal": dict(kind="q4_causal"),
+}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+def weak_scaling_value(units_per_rank: float, world: int, seconds_max: float) -> float:
+    """Whole-job throughput: units all ranks processed / max-over-ranks time."""
+    return units_per_rank * world / seconds_max
+
+
+# ---------------------------------------------------------------- workload
+def make_workload(name: str, rank: int, device):
+    from mla_decode_attention_etap_b200 import workloads as W
+    spec = WORKLOADS[name]
+    seed = 1000 * rank
+    kind = spec.get("kind")
+    if kind == "b64_paged":
+        return W.workload_b64_h16_paged(seed=seed, device=device), "mla_decode_b64_h16_q1_Lunif1to65536_paged64"
+    if kind == "b32_h128":
+        return W.workload_b32_h128_paged(seed=seed, device=device), "mla_decode_b32_h128_q1_Lunif8192to32768_paged64"
+    if kind == "q4_causal":
+        return (W.workload_b16_h16_q4_causal(seed=seed, device=device),
+                "mla_decode_b16_h16_q4_causal_L32768_spikes5pct_x8")
+    w = W.make_workload(spec["batch"], spec["heads"], [spec["seqlen"]] * spec["batch"], seed=seed, device=device)
+    return w, f"mla_decode_b{spec['batch']}_h{spec['heads']}_q1_L{spec['seqlen']}_contiguous"
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained",
+                                                                              pk["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if taken on the current kernel source."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    src = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    if not src or src.group(1) != kernel_source_hash():
+        return None
+    m = re.search(rf"traffic_bytes_per_launch\[{re.escape(workload)}\]:\s*([0-9.eE+]+)", text)
+    return float(m.group(1)) if m else None
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls NVML (SM clock, max clock, throttle reasons) in a thread while the steps run."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting", 0x10: "sync_boost", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.idx, self.period = device_index, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = None
+            try:  # the CUDA device's own UUID: NVML indices ignore CUDA_VISIBLE_DEVICES
+                import torch
+                uuid = str(torch.cuda.get_device_properties(self.idx).uuid)
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        except Exception as e:  # pragma: no cover - NVML missing
+            self.error = repr(e)
+        return self
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception as e:  # pragma: no cover
+                self.error = repr(e)
+                return
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=2)
+        return False
+
+    def summary(self):
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples),
+               "window": "NVML polled every 5 ms from the first warm-up step to the end of the timed steps"}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+# ---------------------------------------------------------------- CPU baseline (oracle)
+def oracle_baseline(w, target_s: float = 12.0):
+    """Time the fp64 oracle on whole sequences of the workload until ~target_s of CPU work."""
+    import numpy as np
+    from mla_decode_attention_etap_b200.workloads import bf16_bits
+    from oracle import mla_oracle as om
+    cores = len(os.sched_getaffinity(0))
+    os.environ["OMP_NUM_THREADS"] = str(cores)
+    om.build()
+    done_bytes, done_flops, t_total, seqs = 0, 0, 0.0, []
+    order = list(range(w.batch))
+    for b in order:
+        L = int(w.seqlens[b])
+        if L == 0:
+            continue
+        rows = w.kv_rows(b).cpu()
+        kv = bf16_bits(rows.reshape(1, L, 576))
+        q = bf16_bits(w.q[b:b + 1].cpu())
+        t0 = time.perf_counter()
+        om.mla_decode(q, kv, np.array([L], np.int32), None, w.softmax_scale, w.causal)
+        t_total += time.perf_counter() - t0
+        done_bytes += L * 1152
+        vis = sum(max((L - w.q_len + t + 1) if w.causal else L, 0) for t in range(w.q_len))
+        done_flops += vis * w.num_heads * 2 * 1088
+        seqs.append(b)
+        if t_total >= target_s:
+            break
+    return {"value": done_bytes / t_total / 1e12, "unit": "TB/s", "cores": cores, "kind": "oracle",
+            "tflops": done_flops / t_total / 1e12,
+            "sample": f"{len(seqs)} whole sequence(s) of the workload (index {seqs[0]}..{seqs[-1]}), "
+                      f"{done_bytes / 1e9:.3f} GB of KV, fp64 C oracle with OpenMP, {t_total:.2f} s"}
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args):
+    """Reference arm: the fp64 oracle on the host, same workload/metric/unit, bounded sample per step."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import torch
+    w, wname = make_workload(args.workload, 0, "cpu")
+    import numpy as np
+    from mla_decode_attention_etap_b200.workloads import bf16_bits
+    from oracle import mla_oracle as om
+    cores = len(os.sched_getaffinity(0))
+    os.environ["OMP_NUM_THREADS"] = str(cores)
+    om.build()
+    # one step = the oracle over a bounded slice of the workload: the first sequence, first 4096 rows
+    b = 0
+    L = min(int(w.seqlens[b]), args.reference_rows)
+    kv = bf16_bits(w.kv_rows(b)[:L].cpu().reshape(1, L, 576))
+    q = bf16_bits(w.q[b:b + 1].cpu())
+    sl = np.array([L], np.int32)
+    for _ in range(args.warmup):
+        om.mla_decode(q, kv, sl, None, w.softmax_scale, w.causal)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        om.mla_decode(q, kv, sl, None, w.softmax_scale, w.causal)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = L * 1152 / dt / 1e12
+    vis = sum(max((L - w.q_len + t + 1) if w.causal else L, 0) for t in range(w.q_len))
+    sample = f"sequence 0, first {L} cache rows, all {w.num_heads} heads x {w.q_len} token(s), per step"
+    line = {"metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "tflops": vis * w.num_heads * 2 * 1088 / dt / 1e12,
+            "config": {"workload": wname, "reference_sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TB/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import mla_decode_attention_etap_b200 as mla
+    from mla_decode_attention_etap_b200 import workloads as W
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    mla.lib()  # fails loudly when the CUDA library is missing
+
+    w, wname = make_workload(args.workload, rank, dev)
+    q, kv, sl = w.q, w.kv, w.seqlens.to(dev)
+    bt = w.block_table.to(dev) if w.block_table is not None else None
+    B, q_len, h = w.batch, w.q_len, w.num_heads
+    dec = mla.MlaDecoder(B, q_len, h, device=dev)
+    o = torch.empty(B, q_len, h, 512, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, q_len, h, dtype=torch.float32, device=dev)
+    seqlens = [int(x) for x in w.seqlens]
+    kv_bytes = W.algorithmic_kv_bytes(seqlens)
+    flops = W.algorithmic_flops(seqlens, q_len, h, w.causal)
+    stream = torch.cuda.current_stream()
+
+    n_events = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_events)]
+
+    def step(i=None):
+        dec.plan(sl)
+        if i is not None:
+            ev[i][0].record(stream)
+        mla.mla_decode_fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o, lse, dec.workspace, dec.n_sms,
+                           mla.FLAG_SKIP_COMBINE)
+        if i is not None:
+            ev[i][1].record(stream)
+        mla.mla_combine(dec.workspace, B, q_len, h, dec.n_sms, o, lse)
+
+    sampler = ClockSampler(local)
+    with sampler:
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(i)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+    status = dec.status()
+    if status != 0:
+        raise RuntimeError(f"device status {mla.STATUS.get(status, status)}")
+    step_s = t_start.elapsed_time(t_end) / 1e3 / args.steps
+    step_s_max = reduce_max(step_s, dev)
+    kern_s = statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3
+    launches = 3 * args.steps  # plan + decode + combine per step
+
+    # ---------------- end to end through the C ABI: pinned host inputs in, outputs back, every step
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    hq = q.cpu().pin_memory()
+    hkv = kv.cpu().pin_memory()
+    hsl = w.seqlens.clone().pin_memory()
+    hbt = w.block_table.clone().pin_memory() if w.block_table is not None else None
+    ho = torch.empty_like(o, device="cpu").pin_memory()
+    hl = torch.empty_like(lse, device="cpu").pin_memory()
+    dq, dkv, dsl = torch.empty_like(q), torch.empty_like(kv), torch.empty_like(sl)
+    dbt = torch.empty_like(bt) if bt is not None else None
+    h2d = hq.numel() * 2 + hkv.numel() * 2 + hsl.numel() * 4 + (hbt.numel() * 4 if hbt is not None else 0)
+    d2h = ho.numel() * 2 + hl.numel() * 4
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dkv.copy_(hkv, non_blocking=True)
+        dsl.copy_(hsl, non_blocking=True)
+        if dbt is not None:
+            dbt.copy_(hbt, non_blocking=True)
+        dec.plan(dsl)
+        mla.mla_decode_fwd(dq, dkv, dsl, dbt, w.softmax_scale, w.causal, o, lse, dec.workspace, dec.n_sms, 0)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_s = reduce_max(e0.elapsed_time(e1) / 1e3 / e2e_steps, dev)
+
+    if rank == 0:
+        hbm_gbs, tc_tflops, tc_sust, peak_src = load_peaks()
+        achieved_gbs = kv_bytes / kern_s / 1e9
+        bound = "hbm" if (kv_bytes / (hbm_gbs * 1e9)) >= (flops / (tc_tflops * 1e12)) else "tensor"
+        if bound == "hbm":
+            roof = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s",
+                    "frac": achieved_gbs / hbm_gbs}
+        else:
+            ach = flops / kern_s / 1e12
+            roof = {"bound": "tensor", "achieved": ach, "peak": tc_tflops, "unit": "TFLOP/s", "frac": ach / tc_tflops}
+        roof["traffic"] = profiled_traffic(wname)
+        roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+        roof["kernel"] = "etap_decode_kernel"
+        roof["kernel_ms"] = kern_s * 1e3
+        roof["tflops"] = flops / kern_s / 1e12
+        roof["algorithmic_bytes_per_launch"] = kv_bytes
+        roof["algorithmic_flops_per_launch"] = flops
+        line = {
+            "metric": METRIC,
+            "value": weak_scaling_value(kv_bytes, world, step_s_max) / 1e12,
+            "unit": "TB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": step_s_max * 1e3,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "tflops": weak_scaling_value(flops, world, step_s_max) / 1e12,
+            "config": {"workload": wname, "batch_per_gpu": B, "heads": h, "q_len": q_len,
+                       "seqlens": (seqlens[0] if len(set(seqlens)) == 1 else
+                                   f"{min(seqlens)}..{max(seqlens)} (mean {sum(seqlens) / len(seqlens):.0f})"),
+                       "d_qk": 576, "d_v": 512, "kv_layout": "paged64" if bt is not None else "contiguous",
+                       "causal": bool(w.causal), "kv_bytes_per_gpu": kv_bytes,
+                       "l2": ("inputs larger than L2 (no flush)" if kv_bytes > 126e6 else
+                              "inputs smaller than L2 (not flushed; numbers are L2-warm)"),
+                       "parallelism": f"dp{world} (independent sequences per GPU, no collective)"},
+            "roofline": roof,
+            "e2e": {"value": weak_scaling_value(kv_bytes, world, e2e_s) / 1e12, "unit": "TB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "ms_per_step": e2e_s * 1e3},
+            "gpu_launches": launches,
+            "clocks": sampler.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_baseline(w, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="b16_h16_64k")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-rows", type=int, default=4096)
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
