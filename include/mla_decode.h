@@ -61,7 +61,8 @@ enum {
     MLA_D_V = 512,       /* value width: the first 512 latent columns */
     MLA_PAGE_SIZE = 64,  /* tokens per page of a paged cache */
     MLA_MAX_BATCH = 65536,
-    MLA_MAX_COLUMNS = 1024 /* max q_len * num_heads */
+    MLA_MAX_COLUMNS = 1024, /* max q_len * num_heads */
+    MLA_STATIC_WORKSPACE_BYTES = 8388608 /* scratch of mla_decode_fwd_static_ws: 8 MiB per GPU */
 };
 
 /* Flags for mla_decode_fwd. */
@@ -144,6 +145,36 @@ MLA_API int mla_decode_read_status(const void *workspace, int *status_out, void 
  */
 MLA_API int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, int num_heads, int num_sms,
                          int32_t *cta_ranges, int32_t *seq_info, int *num_ctas_out, int *num_groups_out);
+
+/*
+ * The whole decode (schedule, ETAP decode, combine) for callers that cannot
+ * allocate device memory: a plugin or extension running inside a host
+ * framework that owns the GPU's memory and hands its guests no allocator, or a
+ * latency-critical serving loop that must not call cudaMalloc/cudaFree because
+ * they can synchronise the whole device. The caller still passes every input
+ * and output; the scratch (schedule + fp32 split partials) lives in one static
+ * device array of MLA_STATIC_WORKSPACE_BYTES inside this library, which every
+ * GPU that loads the library keeps until the process exits. The paper has no
+ * counterpart: this is a deployment convenience.
+ *
+ * Arguments are those of mla_decode_fwd minus the workspace and flags.
+ * Returns MLA_ERR_WORKSPACE, launching nothing, when
+ * mla_decode_workspace_size(batch, q_len, num_heads, num_sms) exceeds
+ * MLA_STATIC_WORKSPACE_BYTES (e.g. B=16, h=16 needs about 5.4 MB on 148 SMs;
+ * B=32, h=128 does not fit). No call allocates memory.
+ *
+ * Set-up: the first call on a device (with that device current) looks up the
+ * array's device address once; make that first call before any stream capture.
+ * Every call shares the one array and it keeps the last call's contents (the
+ * schedule rewrites everything later reads, status word included), so calls
+ * that overlap on the GPU, on different streams or host threads, race: order
+ * them on one stream. The device status word of these calls is internal and
+ * not readable through mla_decode_read_status.
+ */
+MLA_API int mla_decode_fwd_static_ws(const void *q, const void *kv, const int32_t *seqlens,
+                                     const int32_t *block_table, int batch, int q_len, int num_heads,
+                                     int64_t kv_rows, int max_blocks, float softmax_scale, int causal,
+                                     void *o, float *lse, int num_sms, void *stream);
 
 /* Human-readable name of a status code. */
 MLA_API const char *mla_status_string(int status);

@@ -26,7 +26,9 @@ STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3:
           -4: "MLA_ERR_WORKSPACE", -5: "MLA_ERR_CUDA", -6: "MLA_ERR_TIMEOUT", -7: "MLA_ERR_BLOCK_TABLE"}
 
 EXPORTS = ("mla_decode_workspace_size", "mla_decode_plan", "mla_decode_fwd", "mla_combine",
-           "mla_decode_read_status", "mla_decode_plan_host", "mla_status_string", "mla_last_cuda_error")
+           "mla_decode_read_status", "mla_decode_plan_host", "mla_status_string", "mla_last_cuda_error",
+           "mla_decode_fwd_static_ws")
+STATIC_WORKSPACE_BYTES = 8388608
 
 
 class MlaError(RuntimeError):
@@ -63,6 +65,9 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_plan_host.restype = i32
         L.mla_status_string.argtypes = [i32]
         L.mla_status_string.restype = ctypes.c_char_p
+        L.mla_decode_fwd_static_ws.argtypes = [vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp,
+                                               vp, i32, vp]
+        L.mla_decode_fwd_static_ws.restype = i32
         L.mla_last_cuda_error.argtypes = []
         L.mla_last_cuda_error.restype = ctypes.c_char_p
         _lib = L

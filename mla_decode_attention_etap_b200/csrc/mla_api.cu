@@ -270,3 +270,70 @@ int mla_decode_read_status(const void *workspace, int *status_out, void *stream)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Entry point that allocates nothing: the scratch of plan/decode/combine is a
+// file-scope device array (see mla_decode_fwd_static_ws in mla_decode.h).
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_ws[MLA_STATIC_WORKSPACE_BYTES];
+
+std::mutex g_static_ws_mu;
+void *g_static_ws_addr[64] = {};  // device address of g_static_ws, per device, looked up once
+
+// The argument checks of mla_decode_fwd, done before anything is launched.
+int check_static_ws_args(const void *q, const void *kv, const int32_t *seqlens, const int32_t *block_table,
+                         int batch, int q_len, int num_heads, int64_t kv_rows, int max_blocks, float softmax_scale,
+                         int causal, const void *o, const float *lse, int num_sms) {
+    int st = check_shape(batch, q_len, num_heads, num_sms);
+    if (st != MLA_OK) return st;
+    if (!q || !kv || !seqlens || !o || !lse) return MLA_ERR_INVALID_ARG;
+    if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
+    if (kv_rows < 1) return MLA_ERR_INVALID_ARG;
+    if (block_table) {
+        if (kv_rows % MLA_PAGE_SIZE != 0 || max_blocks < 1) return MLA_ERR_INVALID_ARG;
+        if (kv_rows > INT32_MAX) return MLA_ERR_UNSUPPORTED;
+        if (!aligned(block_table, 4)) return MLA_ERR_ALIGNMENT;
+    } else if ((int64_t)batch * kv_rows > INT32_MAX) {
+        return MLA_ERR_UNSUPPORTED;
+    }
+    if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(o, 16) || !aligned(lse, 4) || !aligned(seqlens, 4))
+        return MLA_ERR_ALIGNMENT;
+    if (mla::ws_layout(batch, q_len, num_heads, num_sms).total > (size_t)MLA_STATIC_WORKSPACE_BYTES)
+        return MLA_ERR_WORKSPACE;
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" int mla_decode_fwd_static_ws(const void *q, const void *kv, const int32_t *seqlens,
+                                        const int32_t *block_table, int batch, int q_len, int num_heads,
+                                        int64_t kv_rows, int max_blocks, float softmax_scale, int causal, void *o,
+                                        float *lse, int num_sms, void *stream) {
+    int st = check_static_ws_args(q, kv, seqlens, block_table, batch, q_len, num_heads, kv_rows, max_blocks,
+                                  softmax_scale, causal, o, lse, num_sms);
+    if (st != MLA_OK) return st;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return MLA_ERR_UNSUPPORTED;
+    void *ws = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_static_ws_mu);
+        if (!g_static_ws_addr[dev]) {
+            // In host code g_static_ws names a host-side shadow; the kernels need the device address.
+            void *addr = nullptr;
+            e = cudaGetSymbolAddress(&addr, g_static_ws);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+            g_static_ws_addr[dev] = addr;
+        }
+        ws = g_static_ws_addr[dev];
+    }
+    // The schedule rewrites the header (status word included) and the tables the
+    // decode kernel reads; partial slots are written before the combine reads them.
+    st = mla_decode_plan(seqlens, batch, q_len, num_heads, num_sms, ws, MLA_STATIC_WORKSPACE_BYTES, stream);
+    if (st != MLA_OK) return st;
+    return mla_decode_fwd(q, kv, seqlens, block_table, batch, q_len, num_heads, kv_rows, max_blocks, softmax_scale,
+                          causal, o, lse, ws, MLA_STATIC_WORKSPACE_BYTES, num_sms, 0, stream);
+}
