@@ -12,7 +12,7 @@
 #include <mutex>
 #include <string>
 
-#include "../../include/mla_decode.h"
+#include "mla_decode.h"
 #include "etap_decode_kernel.cuh"
 #include "plan_combine_kernels.cuh"
 #include "plan_core.h"
