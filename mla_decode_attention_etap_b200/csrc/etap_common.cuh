@@ -1,0 +1,202 @@
+// Helpers shared by the ETAP decode kernels: launch parameters, bounded
+// mbarrier waits, the segment iterator over a CTA's flattened tile range, the
+// cross-lane column reduction and bf16 packing.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "plan_core.h"
+#include "ptx_sm100.cuh"
+
+namespace mla {
+
+constexpr int kStatusTimeout = -6;      // MLA_ERR_TIMEOUT
+constexpr int kStatusBlockTable = -7;   // MLA_ERR_BLOCK_TABLE
+constexpr int kStatusInvalid = -1;      // MLA_ERR_INVALID_ARG
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+constexpr uint64_t kDrainLimitNs = 200000000ull;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: p = 2^(x - m) stays <= 256
+
+struct DecodeParams {
+    const int32_t *seqlens;
+    const int32_t *block_table;
+    int32_t *ws;  // workspace (int32 view)
+    float *opart;
+    float *lsepart;
+    __nv_bfloat16 *o;
+    float *lse;
+    int64_t kv_rows;  // contiguous: rows per sequence; paged: total rows of the pool
+    int batch, q_len, num_heads, ncols, ctas, groups, max_blocks, paged, causal;
+    float scale_log2;  // softmax_scale * log2(e)
+    int cta_ranges_off, tile_off_off, seq_info_off;  // int32 offsets into ws
+};
+
+// Bounded wait on an mbarrier phase.  Returns false (and raises the CTA abort
+// flag) when the wait ran past kWaitLimitNs, or when another role aborted.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                           int32_t *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((spin & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicCAS(status, 0, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+// Wait used only while draining after an abort: bounded, ignores the abort flag.
+__device__ __forceinline__ void drain_phase(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kDrainLimitNs) return;
+    }
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Walks the (sequence, tile range) segments of flattened tiles [fb, fe).
+struct SegIter {
+    int64_t f, fe;
+    int b;
+    __device__ void init(const int32_t *tile_off, int batch, int64_t fb, int64_t fe_) {
+        f = fb;
+        fe = fe_;
+        // last b with tile_off[b] <= fb
+        int lo = 0, hi = batch;  // tile_off[batch] = total > fb when fb < fe
+        while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if (tile_off[mid] <= fb) lo = mid; else hi = mid;
+        }
+        b = lo;
+    }
+    __device__ bool next(const int32_t *tile_off, int &ob, int &t0, int &t1) {
+        if (f >= fe) return false;
+        while (tile_off[b + 1] <= f) ++b;
+        ob = b;
+        t0 = (int)(f - tile_off[b]);
+        int64_t e = fe < (int64_t)tile_off[b + 1] ? fe : (int64_t)tile_off[b + 1];
+        t1 = (int)(e - tile_off[b]);
+        f = e;
+        return true;
+    }
+};
+
+// Tile-by-tile cursor over the same segments (the MMA issuer keeps one for
+// the scores and one for the output contraction).
+struct TileCursor {
+    SegIter it;
+    int b, t0, t, t1;
+    bool valid;
+    __device__ void init(const int32_t *tile_off, int batch, int64_t fb, int64_t fe) {
+        it.init(tile_off, batch, fb, fe);
+        b = t0 = t = t1 = 0;
+        valid = it.next(tile_off, b, t0, t1);
+        t = t0;
+    }
+    __device__ void advance(const int32_t *tile_off) {
+        if (t + 1 < t1) {
+            ++t;
+            return;
+        }
+        valid = it.next(tile_off, b, t0, t1);
+        t = t0;
+    }
+    __device__ bool first() const { return t == t0; }
+    __device__ bool last() const { return t == t1 - 1; }
+};
+
+// Column reduction of 16 values per lane across the 32 lanes of a warp
+// (recursive halving: 16 shuffles instead of 5 per column).  Lane l ends with
+// the reduction of column col16(l); lanes l and l^1 hold the same column.
+__device__ __forceinline__ int col16(int lane) {
+    return (((lane >> 4) & 1) << 3) | (((lane >> 3) & 1) << 2) | (((lane >> 2) & 1) << 1) | ((lane >> 1) & 1);
+}
+template <bool IS_MAX>
+__device__ __forceinline__ float op2(float a, float b) {
+    return IS_MAX ? fmaxf(a, b) : a + b;
+}
+template <bool IS_MAX>
+__device__ __forceinline__ float warp_colreduce16(const float (&v)[16], int lane) {
+    float a8[8], a4[4], a2[2];
+    bool up = (lane & 16) != 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float send = up ? v[j] : v[j + 8];
+        float keep = up ? v[j + 8] : v[j];
+        a8[j] = op2<IS_MAX>(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+    }
+    up = (lane & 8) != 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float send = up ? a8[j] : a8[j + 4];
+        float keep = up ? a8[j + 4] : a8[j];
+        a4[j] = op2<IS_MAX>(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+    }
+    up = (lane & 4) != 0;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        float send = up ? a4[j] : a4[j + 2];
+        float keep = up ? a4[j + 2] : a4[j];
+        a2[j] = op2<IS_MAX>(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+    }
+    up = (lane & 2) != 0;
+    float a1 = op2<IS_MAX>(up ? a2[1] : a2[0], __shfl_xor_sync(0xffffffffu, up ? a2[0] : a2[1], 2));
+    return op2<IS_MAX>(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Spinning variants for the softmax warps: a non-blocking probe in a loop
+// resumes the moment the phase completes (a suspended try_wait can wake late,
+// and the slowest of the 128 threads sets the pace of the next named barrier).
+template <bool CLUSTER>
+__device__ __forceinline__ bool spin_phase(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                           int32_t *status) {
+    auto probe = [&]() { return CLUSTER ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity); };
+    if (probe()) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (probe()) return true;
+        if ((spin & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicCAS(status, 0, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait on a phase completed by the peer CTA of the cluster (acquire at cluster scope).
+__device__ __forceinline__ bool wait_phase_cluster(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                                   int32_t *status) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((spin & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicCAS(status, 0, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+}  // namespace mla

@@ -1,0 +1,705 @@
+// ETAP decode kernel on a pair of SMs (a 2-CTA cluster), sm_100a.
+//
+// Computation (FlashMLA-ETAP technical summary, "Methodology", ETAP steps 1-4):
+// S^T = K Q^T with the 128 KV rows of a tile as the UMMA M dimension and the
+// query columns (heads x tokens) as N; P^T = softmax(S^T) down each column;
+// O^T = V^T P^T; O = (O^T)^T.  "Integration and Implementation" describes a
+// producer that streams KV from HBM into a circular shared-memory buffer and
+// consumers that compute the scores and the softmax statistics block by block;
+// this kernel keeps those roles but lays them out for Blackwell:
+//
+//   * The two CTAs of a cluster split every KV row by latent columns: rank r
+//     holds value columns 256r..256r+255 and rope columns 512+32r..512+32r+31.
+//     A 128-row tile then needs 72 KB of shared memory per CTA instead of
+//     144 KB, so each CTA's ring keeps ~2.5 tiles in flight and
+//     the loads of tile k+1 overlap the softmax and the second contraction of
+//     tile k.  Each CTA computes a partial S^T over its own columns; the 128
+//     softmax threads send their rows of it to the peer CTA (st.async into the
+//     peer's shared memory, counted on the peer's mbarrier) and add the peer's
+//     rows, so both CTAs hold the same S^T (fp32 addition commutes), run the
+//     same softmax and each accumulates O^T for its own 256 value columns.
+//   * warp 0: TMA producer (Q once per segment, KV tiles into 32 KB slots of
+//     two 64-column chunks plus an 8 KB slot for the 32 rope columns; tail
+//     rows zeroed);
+//   * warp 1 lane 0: tcgen05.mma issuer, S^T of tile k+1 before O^T of tile k;
+//   * warps 2..5: one TMEM lane (= one KV row) per thread; the column softmax
+//     reduces ACROSS threads; P^T goes to shared memory as bf16 hi | lo.
+//
+// Every wait is bounded; see etap_common.cuh.
+#pragma once
+
+#include "etap_common.cuh"
+
+namespace mla {
+
+__host__ __device__ constexpr uint32_t align1024(uint32_t x) { return (x + 1023u) & ~1023u; }
+__host__ __device__ constexpr uint32_t pow2_at_least(uint32_t x) {
+    return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512;
+}
+
+// NG query columns per cluster; NV V-pair slots, NR rope slots, PB P^T buffers per CTA.
+template <int NG_, int NV_, int NR_, int PB_>
+struct PairCfg {
+    static constexpr int NG = NG_;
+    static constexpr int NP = 2 * NG;  // UMMA N of step 3: [P_hi | P_lo]
+    static constexpr int CH = NG / 16;  // 16-column chunks of softmax and exchange
+    static constexpr int NV = NV_, NR = NR_, PB = PB_;
+    static constexpr int PAIRS = 2;                                    // V pairs of a tile in one CTA
+    static constexpr int EARLY = (NV - PAIRS) < PAIRS ? (NV - PAIRS) : PAIRS;  // pairs of tile k+1 free of tile k
+    static constexpr int XS = 2;                                       // exchange slots
+    static constexpr uint32_t CHUNK = 16384;                           // 128 rows x 64 bf16, 128B swizzle
+    static constexpr uint32_t HALF = 8192;                             // 64 rows of a chunk = one TMA box
+    static constexpr uint32_t V_SLOT = 2 * CHUNK;
+    static constexpr uint32_t R_SLOT = 128 * 64;                       // 128 rows x 32 rope bf16, 64B swizzle
+    static constexpr uint32_t R_HALF = 64 * 64;                        // 64 rows of it = one TMA box
+    static constexpr uint32_t Q_CHUNK = NG * 128;                      // NG rows x 64 columns
+    static constexpr uint32_t Q_ROPE = NG * 64;                        // NG rows x 32 rope columns
+    static constexpr int AW = NP < 64 ? NP : 64;                       // P^T swizzle atom width (columns)
+    static constexpr int NA = NP / AW;                                 // atoms along N
+    static constexpr uint32_t P_PITCH = AW * 2;                        // bytes per KV row inside an atom
+    static constexpr uint32_t P_ATOM = 128 * P_PITCH;
+    static constexpr uint32_t P_BUF = NA * P_ATOM;
+    static constexpr uint32_t P_SWIZZLE = (P_PITCH == 128) ? kSwizzle128B : kSwizzle64B;
+    static constexpr uint32_t P_SWZ_MASK = (P_PITCH == 128) ? 7u : 3u;
+    static constexpr uint32_t X_SLOT = 128 * 16 * 4;                   // 128 rows x 16 fp32 partial scores
+    static constexpr uint32_t OFF_V = 0;
+    static constexpr uint32_t OFF_R = OFF_V + NV * V_SLOT;
+    static constexpr uint32_t OFF_Q = OFF_R + NR * R_SLOT;
+    static constexpr uint32_t OFF_QR = OFF_Q + 4 * Q_CHUNK;
+    static constexpr uint32_t OFF_P = align1024(OFF_QR + Q_ROPE);
+    static constexpr uint32_t OFF_X = OFF_P + PB * P_BUF;
+    static constexpr uint32_t OFF_BAR = OFF_X + XS * X_SLOT;
+    static constexpr uint32_t OFF_RED = OFF_BAR + 512;                 // float [2][4][16] column max exchange
+    static constexpr uint32_t OFF_REDL = OFF_RED + 512;                // float [4][NG] column sum exchange
+    static constexpr uint32_t OFF_MISC = OFF_REDL + 16 * NG;
+    static constexpr uint32_t BYTES = OFF_MISC + 64;
+    static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;               // slack for 1024-byte alignment
+    static constexpr uint32_t O_COL = 0;                               // 2 M-tiles x NP columns
+    static constexpr uint32_t S_COL = 2 * NP;                          // 2 buffers x NG columns
+    static constexpr uint32_t TMEM_COLS = pow2_at_least(2 * NP + 2 * NG);
+    static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, NG, 0, 0);
+    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, NP, 1, 1);
+};
+
+using PairCfg16 = PairCfg<16, 5, 2, 2>;  // h*q_len <= 16
+using PairCfg64 = PairCfg<64, 3, 2, 1>;  // 16 < h*q_len, in groups of 64 columns
+
+static_assert(PairCfg16::SMEM_ALLOC <= 232448 && PairCfg64::SMEM_ALLOC <= 232448, "shared memory plan > 227 KB");
+static_assert(PairCfg16::TMEM_COLS <= 512 && PairCfg64::TMEM_COLS <= 512, "TMEM plan");
+static_assert(PairCfg16::OFF_P % 1024 == 0 && PairCfg64::OFF_P % 1024 == 0, "alignment");
+static_assert(PairCfg16::OFF_QR % 512 == 0 && PairCfg64::OFF_QR % 512 == 0, "alignment");
+
+template <class C>
+struct PairBars {
+    static constexpr int VFULL = 0;
+    static constexpr int VEMPTY = VFULL + C::NV;
+    static constexpr int RFULL = VEMPTY + C::NV;
+    static constexpr int REMPTY = RFULL + C::NR;
+    static constexpr int QFULL = REMPTY + C::NR;
+    static constexpr int QEMPTY = QFULL + 1;
+    static constexpr int SFULL = QEMPTY + 1;
+    static constexpr int SEMPTY = SFULL + 2;
+    static constexpr int PFULL = SEMPTY + 2;
+    static constexpr int PEMPTY = PFULL + C::PB;
+    static constexpr int TAIL = PEMPTY + C::PB;
+    static constexpr int FINAL = TAIL + 1;
+    static constexpr int RED = FINAL + 1;
+    static constexpr int REDL = RED + 1;
+    static constexpr int XFULL = REDL + 1;
+    static constexpr int COUNT = XFULL + C::XS;
+};
+static_assert(PairBars<PairCfg16>::COUNT * 8 <= 512 && PairBars<PairCfg64>::COUNT * 8 <= 512, "barrier area");
+
+// Byte offset of 16-byte chunk j of row r in a row-major buffer of `pitch`-byte
+// rows swizzled like the MMA operand (chunk index XOR address bits 7+).
+__device__ __forceinline__ uint32_t swz_off(uint32_t r, uint32_t j, uint32_t pitch, uint32_t mask) {
+    const uint32_t off = r * pitch;
+    return off + ((j ^ ((off >> 7) & mask)) << 4);
+}
+
+template <class C>
+__global__ void __launch_bounds__(192, 1)
+    etap_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                     const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_kvr,
+                     const __grid_constant__ DecodeParams p) {
+    using BR = PairBars<C>;
+    constexpr int NG = C::NG;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_addr(smem_raw);
+    const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+    uint8_t *smem = smem_raw + (sbase - raw_addr);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const uint32_t peer = rank ^ 1u;
+    const int cluster = blockIdx.x >> 1;
+    const int unit = cluster / p.groups;
+    const int grp = cluster % p.groups;
+    int32_t *status = p.ws + kHdrStatus;
+
+    // The schedule must come from a plan for this same grid (uniform in the whole cluster).
+    const bool plan_ok = p.ws[kHdrCtas] == p.ctas && p.ws[kHdrGroups] == p.groups && p.ws[kHdrBatch] == p.batch;
+
+    auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * (uint32_t)i; };
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::NV; ++i) {
+            mbar_init(bar(BR::VFULL + i), 1);
+            mbar_init(bar(BR::VEMPTY + i), 1);
+        }
+        for (int i = 0; i < C::NR; ++i) {
+            mbar_init(bar(BR::RFULL + i), 1);
+            mbar_init(bar(BR::REMPTY + i), 1);
+        }
+        mbar_init(bar(BR::QFULL), 1);
+        mbar_init(bar(BR::QEMPTY), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(BR::SFULL + i), 1);
+            mbar_init(bar(BR::SEMPTY + i), 4);
+        }
+        for (int i = 0; i < C::PB; ++i) {
+            mbar_init(bar(BR::PFULL + i), 4);
+            mbar_init(bar(BR::PEMPTY + i), 1);
+        }
+        mbar_init(bar(BR::TAIL), 1);
+        mbar_init(bar(BR::FINAL), 1);
+        mbar_init(bar(BR::RED), 4);
+        mbar_init(bar(BR::REDL), 4);
+        for (int i = 0; i < C::XS; ++i) mbar_init(bar(BR::XFULL + i), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_kv);
+        tma_prefetch_desc(&tm_qr);
+        tma_prefetch_desc(&tm_kvr);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers are initialised before any remote arrive or st.async
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int32_t *ranges = p.ws + p.cta_ranges_off;
+    const int32_t *tile_off = p.ws + p.tile_off_off;
+    const int32_t *seq_info = p.ws + p.seq_info_off;
+    const int64_t fb = plan_ok ? ranges[2 * unit] : 0, fe = plan_ok ? ranges[2 * unit + 1] : 0;
+    if (!plan_ok && threadIdx.x == 0) atomicCAS(status, 0, kStatusInvalid);
+    const int64_t l_cap = p.paged ? (int64_t)p.max_blocks * kPage : p.kv_rows;
+    const int rope_x = 512 + 32 * (int)rank;  // first rope column of this CTA
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int phases_v[C::NV], arms_r[C::NR];
+        bool tma_v[C::NV];
+#pragma unroll
+        for (int i = 0; i < C::NV; ++i) {
+            phases_v[i] = 0;
+            tma_v[i] = false;
+        }
+#pragma unroll
+        for (int i = 0; i < C::NR; ++i) arms_r[i] = 0;
+        int arms_q = 0, tail_uses = 0;
+        bool ok = true;
+        if (fb < fe) {
+            SegIter it;
+            it.init(tile_off, p.batch, fb, fe);
+            int b, t0, t1, seg = 0, k = 0;
+            while (ok && it.next(tile_off, b, t0, t1)) {
+                int L = p.seqlens[b];
+                if ((int64_t)L > l_cap) {
+                    if (lane == 0) atomicCAS(status, 0, kStatusInvalid);
+                    L = (int)l_cap;
+                }
+                if (L < 0) L = 0;
+                if (seg > 0) ok = wait_phase(bar(BR::QEMPTY), (seg - 1) & 1, abort_flag, status);
+                if (!ok) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar(BR::QFULL), 4 * C::Q_CHUNK + C::Q_ROPE);
+                    const int qrow = b * p.ncols + grp * NG;
+                    for (int j = 0; j < 4; ++j)
+                        tma_load_2d(sbase + C::OFF_Q + j * C::Q_CHUNK, &tm_q, bar(BR::QFULL), (4 * (int)rank + j) * 64,
+                                    qrow);
+                    tma_load_2d(sbase + C::OFF_QR, &tm_qr, bar(BR::QFULL), rope_x, qrow);
+                }
+                ++arms_q;
+                for (int t = t0; t < t1 && ok; ++t, ++k) {
+                    const int row0 = t * kTileRows;
+                    int valid = L - row0;
+                    valid = valid < 0 ? 0 : (valid > kTileRows ? kTileRows : valid);
+                    int y[2];
+                    bool loaded[2];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        loaded[hh] = valid > 64 * hh;
+                        y[hh] = 0;
+                        if (loaded[hh]) {
+                            if (p.paged) {
+                                const int blk = p.block_table[(int64_t)b * p.max_blocks + (row0 >> 6) + hh];
+                                if (blk < 0 || (int64_t)blk * kPage >= p.kv_rows) {
+                                    if (lane == 0) atomicCAS(status, 0, kStatusBlockTable);
+                                    loaded[hh] = false;
+                                } else {
+                                    y[hh] = blk * kPage;
+                                }
+                            } else {
+                                y[hh] = (int)((int64_t)b * p.kv_rows + row0 + 64 * hh);
+                            }
+                        }
+                    }
+                    const int nload = (int)loaded[0] + (int)loaded[1];
+                    const bool tail = !(loaded[0] && loaded[1] && valid == kTileRows);
+                    {
+                        // this CTA's 32 rope columns: rows past the end are masked in S^T, no zeroing needed
+                        const int rs = k % C::NR;
+                        ok = wait_phase(bar(BR::REMPTY + rs), ((k / C::NR) & 1) ^ 1, abort_flag, status);
+                        if (!ok) break;
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(bar(BR::RFULL + rs), nload * C::R_HALF);
+                            for (int hh = 0; hh < 2; ++hh)
+                                if (loaded[hh])
+                                    tma_load_2d(sbase + C::OFF_R + rs * C::R_SLOT + hh * C::R_HALF, &tm_kvr,
+                                                bar(BR::RFULL + rs), rope_x, y[hh]);
+                        }
+                        ++arms_r[rs];
+                    }
+                    for (int i = 0; i < C::PAIRS && ok; ++i) {
+                        const int g2 = C::PAIRS * k + i;
+                        const int vs = g2 % C::NV;
+                        const int c0 = 4 * (int)rank + 2 * i;  // latent chunks c0, c0+1 of this CTA's half
+                        ok = wait_phase(bar(BR::VEMPTY + vs), ((g2 / C::NV) & 1) ^ 1, abort_flag, status);
+                        if (!ok) break;
+                        const uint32_t dst = sbase + C::OFF_V + vs * C::V_SLOT;
+                        if (!tail) {
+                            if (lane == 0) {
+                                mbar_arrive_expect_tx(bar(BR::VFULL + vs), C::V_SLOT);
+                                for (int hc = 0; hc < 2; ++hc)
+                                    for (int hh = 0; hh < 2; ++hh)
+                                        tma_load_2d(dst + hc * C::CHUNK + hh * C::HALF, &tm_kv, bar(BR::VFULL + vs),
+                                                    (c0 + hc) * 64, y[hh]);
+                            }
+                            ++phases_v[vs];
+                            tma_v[vs] = true;
+                        } else {
+                            // tail tile: land the valid rows, zero all others so whatever the cache holds
+                            // past L_b (NaN included) meets P = 0 as an exact 0
+                            if (nload > 0) {
+                                if (lane == 0) {
+                                    mbar_arrive_expect_tx(bar(BR::TAIL), 2 * nload * C::HALF);
+                                    for (int hc = 0; hc < 2; ++hc)
+                                        for (int hh = 0; hh < 2; ++hh)
+                                            if (loaded[hh])
+                                                tma_load_2d(dst + hc * C::CHUNK + hh * C::HALF, &tm_kv, bar(BR::TAIL),
+                                                            (c0 + hc) * 64, y[hh]);
+                                }
+                                ok = wait_phase(bar(BR::TAIL), tail_uses & 1, abort_flag, status);
+                                ++tail_uses;
+                                if (!ok) break;
+                            }
+                            for (int idx = lane; idx < 2 * kTileRows * 8; idx += 32) {
+                                const int hc = idx / (kTileRows * 8);
+                                const int r = (idx / 8) % kTileRows;
+                                const int c16 = idx % 8;
+                                if (r < valid && loaded[r >> 6]) continue;
+                                *reinterpret_cast<uint4 *>(smem + C::OFF_V + vs * C::V_SLOT + hc * C::CHUNK + r * 128 +
+                                                           c16 * 16) = make_uint4(0u, 0u, 0u, 0u);
+                            }
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar(BR::VFULL + vs));
+                            ++phases_v[vs];
+                            tma_v[vs] = false;
+                        }
+                    }
+                }
+                ++seg;
+            }
+        }
+        if (!ok) {
+            for (int i = 0; i < C::NV; ++i)
+                if (tma_v[i]) drain_phase(bar(BR::VFULL + i), (phases_v[i] - 1) & 1);
+            for (int i = 0; i < C::NR; ++i)
+                if (arms_r[i] > 0) drain_phase(bar(BR::RFULL + i), (arms_r[i] - 1) & 1);
+            if (arms_q > 0) drain_phase(bar(BR::QFULL), (arms_q - 1) & 1);
+            if (tail_uses > 0) drain_phase(bar(BR::TAIL), (tail_uses - 1) & 1);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        // An event loop: step 1 of the next tile goes as soon as its KV and Q are
+        // in shared memory, step 3 of the oldest pending tile as soon as its P^T
+        // is; "S^T ready" is committed right after the scores' MMAs, so the
+        // softmax of tile k overlaps step 3 of tile k-1 on the tensor pipe.
+        if (lane == 0 && fb < fe) {
+            const uint32_t q_base = sbase + C::OFF_Q;
+            auto qk_chunk = [&](uint32_t d_s, uint32_t a_base, int qchunk, bool init) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint64_t a = smem_desc(a_base + 32u * j, 16, 1024, kSwizzle128B);
+                    const uint64_t bq = smem_desc(q_base + qchunk * C::Q_CHUNK + 32u * j, 16, 1024, kSwizzle128B);
+                    umma_bf16(d_s, a, bq, C::IDESC_QK, (init && j == 0) ? 0u : 1u);
+                }
+            };
+            TileCursor qc, pc;
+            qc.init(tile_off, p.batch, fb, fe);
+            pc.init(tile_off, p.batch, fb, fe);
+            int kq = 0, kp = 0, seg_q = 0;
+            uint64_t t_last = global_timer_ns();
+            while (pc.valid) {
+                bool progressed = false;
+                if (qc.valid) {
+                    const int rs = kq % C::NR;
+                    bool ready = mbar_test_wait(bar(BR::SEMPTY + (kq & 1)), ((kq >> 1) & 1) ^ 1);
+                    if (ready && qc.first()) ready = mbar_test_wait(bar(BR::QFULL), seg_q & 1);
+                    if (ready) ready = mbar_test_wait(bar(BR::RFULL + rs), (kq / C::NR) & 1);
+                    for (int i = 0; i < C::PAIRS && ready; ++i) {
+                        const int g2 = C::PAIRS * kq + i;
+                        ready = mbar_test_wait(bar(BR::VFULL + g2 % C::NV), (g2 / C::NV) & 1);
+                    }
+                    if (ready) {
+                        tc_fence_after();
+                        const uint32_t d_s = tmem + C::S_COL + (kq & 1) * NG;
+                        // 32 rope columns (K-major, 64-byte rows): two K-steps; the first (re)initialises S^T
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const uint64_t a = smem_desc(sbase + C::OFF_R + rs * C::R_SLOT + 32u * j, 16, 512, kSwizzle64B);
+                            const uint64_t bq = smem_desc(sbase + C::OFF_QR + 32u * j, 16, 512, kSwizzle64B);
+                            umma_bf16(d_s, a, bq, C::IDESC_QK, j == 0 ? 0u : 1u);
+                        }
+                        umma_commit(bar(BR::REMPTY + rs));
+                        for (int i = 0; i < C::PAIRS; ++i) {
+                            const int g2 = C::PAIRS * kq + i;
+                            const uint32_t slot = sbase + C::OFF_V + (g2 % C::NV) * C::V_SLOT;
+                            qk_chunk(d_s, slot, 2 * i, false);
+                            qk_chunk(d_s, slot + C::CHUNK, 2 * i + 1, false);
+                        }
+                        umma_commit(bar(BR::SFULL + (kq & 1)));
+                        if (qc.last()) {
+                            umma_commit(bar(BR::QEMPTY));
+                            ++seg_q;
+                        }
+                        qc.advance(tile_off);
+                        ++kq;
+                        progressed = true;
+                    }
+                }
+                if (kp < kq) {
+                    const int pb = kp % C::PB;
+                    if (mbar_test_wait(bar(BR::PFULL + pb), (kp / C::PB) & 1)) {
+                        tc_fence_after();
+                        const bool first = pc.first();
+                        const uint32_t p_base = sbase + C::OFF_P + pb * C::P_BUF;
+                        for (int i = 0; i < C::PAIRS; ++i) {
+                            const int g2 = C::PAIRS * kp + i;
+                            const int vs = g2 % C::NV;
+                            const uint32_t v_base = sbase + C::OFF_V + vs * C::V_SLOT;
+                            const uint32_t d_o = tmem + C::O_COL + i * C::NP;
+#pragma unroll
+                            for (int s = 0; s < 8; ++s) {
+                                // A = V^T: M = 128 latent columns (two chunks CHUNK apart), K = 16 KV rows (MN-major)
+                                const uint64_t a = smem_desc(v_base + 2048u * s, C::CHUNK, 1024, kSwizzle128B);
+                                // B = [P_hi | P_lo]^T: K = 16 KV rows, N = NP columns (MN-major)
+                                const uint64_t bp = smem_desc(p_base + 16u * C::P_PITCH * s, C::P_ATOM,
+                                                              8 * C::P_PITCH, C::P_SWIZZLE);
+                                umma_bf16(d_o, a, bp, C::IDESC_PV, (first && s == 0) ? 0u : 1u);
+                            }
+                            umma_commit(bar(BR::VEMPTY + vs));
+                        }
+                        umma_commit(bar(BR::PEMPTY + pb));
+                        pc.advance(tile_off);
+                        ++kp;
+                        progressed = true;
+                    }
+                }
+                if (progressed) {
+                    t_last = global_timer_ns();
+                } else if (*abort_flag) {
+                    break;
+                } else if (global_timer_ns() - t_last > kWaitLimitNs) {
+                    *abort_flag = 1;
+                    atomicCAS(status, 0, kStatusTimeout);
+                    break;
+                }
+            }
+            umma_commit(bar(BR::FINAL));
+            drain_phase(bar(BR::FINAL), 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue (warps 2..5)
+        // The four warps synchronise through named barrier 1; a failed (timed
+        // out) wait only clears this thread's `ok`, and the next bar.red turns
+        // that into a uniform stop, so no thread is left waiting at a barrier.
+        constexpr uint32_t SMX = 1, NSM = 128;
+        const int quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        float *red = reinterpret_cast<float *>(smem + C::OFF_RED);    // [2][4][16]
+        float *redl = reinterpret_cast<float *>(smem + C::OFF_REDL);  // [4][NG]
+        const uint32_t x_remote = map_to_rank(sbase + C::OFF_X, peer);
+        const uint32_t xfull_remote = map_to_rank(bar(BR::XFULL), peer);
+        bool ok = true, stop = false;
+        if (fb < fe) {
+            SegIter it;
+            it.init(tile_off, p.batch, fb, fe);
+            int b, t0, t1, k = 0, seg = 0, e = 0, red_uses = 0;
+            while (!stop && it.next(tile_off, b, t0, t1)) {
+                int L = p.seqlens[b];
+                if ((int64_t)L > l_cap) L = (int)l_cap;
+                if (L < 0) L = 0;
+                float m[NG], lpart[NG];
+#pragma unroll
+                for (int n = 0; n < NG; ++n) {
+                    m[n] = -INFINITY;
+                    lpart[n] = 0.f;
+                }
+                for (int t = t0; t < t1 && !stop; ++t, ++k) {
+                    const bool first = (t == t0);
+                    const int pb = k % C::PB;
+                    ok = ok && spin_phase<false>(bar(BR::SFULL + (k & 1)), (k >> 1) & 1, abort_flag, status);
+                    tc_fence_after();
+                    const int rg = t * kTileRows + row;
+                    // every row of the tile visible to every column: no per-column mask needed
+                    const bool full_tile = (t + 1) * kTileRows <= (p.causal ? L - p.q_len + 1 : L);
+                    bool waited_prev = false, rescale_any = false;
+#pragma unroll
+                    for (int ch = 0; ch < C::CH; ++ch) {
+                        float x[16];
+                        tmem_ld16(tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch, x);
+                        tmem_wait_ld();
+                        if (ch == C::CH - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(bar(BR::SEMPTY + (k & 1)));
+                        }
+                        // ---- exchange of the partial scores with the peer CTA.  Slot xs is free for
+                        // exchange e without a handshake: the peer overwrites it (exchange e + XS) only
+                        // after receiving our exchange e + XS - 1, which we send after consuming e.
+                        static_assert(C::XS >= 2, "slot reuse relies on at least two exchange slots");
+                        const int xs = e % C::XS, xu = e / C::XS;
+                        ++e;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            st_async_v4(x_remote + xs * C::X_SLOT + swz_off(row, j, 64, 3), __float_as_uint(x[4 * j]),
+                                        __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
+                                        __float_as_uint(x[4 * j + 3]), xfull_remote + 8u * xs);
+                        if (row == 0) mbar_arrive_expect_tx(bar(BR::XFULL + xs), C::X_SLOT);
+                        ok = ok && spin_phase<true>(bar(BR::XFULL + xs), xu & 1, abort_flag, status);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float4 v = *reinterpret_cast<const float4 *>(smem + C::OFF_X + xs * C::X_SLOT +
+                                                                               swz_off(row, j, 64, 3));
+                            x[4 * j] += v.x;
+                            x[4 * j + 1] += v.y;
+                            x[4 * j + 2] += v.z;
+                            x[4 * j + 3] += v.w;
+                        }
+                        // ---- scale + mask
+                        if (full_tile) {
+#pragma unroll
+                            for (int n = 0; n < 16; ++n) x[n] *= p.scale_log2;
+                        } else {
+#pragma unroll
+                            for (int n = 0; n < 16; ++n) {
+                                const int ng = grp * NG + 16 * ch + n;
+                                int vis = 0;
+                                if (ng < p.ncols) {
+                                    vis = p.causal ? (L - p.q_len + ng / p.num_heads + 1) : L;
+                                    vis = vis < 0 ? 0 : vis;
+                                }
+                                x[n] = (rg < vis) ? x[n] * p.scale_log2 : -INFINITY;
+                            }
+                        }
+                        // ---- running maximum: kept unless some row of the tile exceeds it by > 2^8
+                        bool need = first || !ok;
+#pragma unroll
+                        for (int n = 0; n < 16; ++n) need = need || (x[n] > m[16 * ch + n] + kRescaleThreshold);
+                        float alpha[16];
+#pragma unroll
+                        for (int n = 0; n < 16; ++n) alpha[n] = 1.f;
+                        bool rescale = false;
+                        if (named_bar_or(SMX, NSM, need)) {
+                            if (!named_bar_and(SMX, NSM, ok)) {
+                                stop = true;
+                                break;
+                            }
+                            // column maximum of the tile: across lanes, then across the 4 warps
+                            const float wmax = warp_colreduce16<true>(x, lane);
+                            float *rb = red + (red_uses & 1) * 64;
+                            ++red_uses;
+                            if ((lane & 1) == 0) rb[quad * 16 + col16(lane)] = wmax;
+                            named_bar_sync(SMX, NSM);
+#pragma unroll
+                            for (int n4 = 0; n4 < 16; n4 += 4) {
+                                const float4 a = *reinterpret_cast<const float4 *>(rb + 0 * 16 + n4);
+                                const float4 bq = *reinterpret_cast<const float4 *>(rb + 1 * 16 + n4);
+                                const float4 c = *reinterpret_cast<const float4 *>(rb + 2 * 16 + n4);
+                                const float4 d = *reinterpret_cast<const float4 *>(rb + 3 * 16 + n4);
+                                const float mt4[4] = {fmaxf(fmaxf(a.x, bq.x), fmaxf(c.x, d.x)),
+                                                      fmaxf(fmaxf(a.y, bq.y), fmaxf(c.y, d.y)),
+                                                      fmaxf(fmaxf(a.z, bq.z), fmaxf(c.z, d.z)),
+                                                      fmaxf(fmaxf(a.w, bq.w), fmaxf(c.w, d.w))};
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    const int n = n4 + u, cn = 16 * ch + n;
+                                    if (first) {
+                                        m[cn] = mt4[u];
+                                    } else if (mt4[u] > m[cn] + kRescaleThreshold) {
+                                        alpha[n] = fast_exp2(m[cn] - mt4[u]);
+                                        m[cn] = mt4[u];
+                                        rescale = true;
+                                    }
+                                }
+                            }
+                        }
+                        float pv[16];
+#pragma unroll
+                        for (int n = 0; n < 16; ++n) {
+                            const int cn = 16 * ch + n;
+                            const float mu = (m[cn] == -INFINITY) ? 0.f : m[cn];
+                            pv[n] = fast_exp2(x[n] - mu);
+                            lpart[cn] = lpart[cn] * alpha[n] + pv[n];
+                        }
+                        // ---- P^T row chunk -> shared memory: bf16 hi into columns [16ch, 16ch+16), lo into NG + that
+                        if (ch == 0)
+                            ok = ok && spin_phase<false>(bar(BR::PEMPTY + pb), ((k / C::PB) & 1) ^ 1, abort_flag, status);
+                        {
+                            uint32_t hi[8], lo[8];
+#pragma unroll
+                            for (int n = 0; n < 16; n += 2) {
+                                const __nv_bfloat16 h0 = __float2bfloat16_rn(pv[n]);
+                                const __nv_bfloat16 h1 = __float2bfloat16_rn(pv[n + 1]);
+                                hi[n / 2] =
+                                    (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+                                lo[n / 2] = pack_bf16x2(pv[n] - __bfloat162float(h0), pv[n + 1] - __bfloat162float(h1));
+                            }
+                            uint8_t *pbuf = smem + C::OFF_P + pb * C::P_BUF;
+#pragma unroll
+                            for (int half = 0; half < 2; ++half) {
+                                const uint32_t *w = half == 0 ? hi : lo;
+                                const int col0 = half * NG + 16 * ch;  // first P^T column of these 16
+                                const int atom = col0 / C::AW;
+                                const int j0 = (col0 % C::AW) / 8;  // 16-byte chunk within the atom row
+#pragma unroll
+                                for (int jj = 0; jj < 2; ++jj) {
+                                    uint4 *dst = reinterpret_cast<uint4 *>(
+                                        pbuf + atom * C::P_ATOM + swz_off(row, j0 + jj, C::P_PITCH, C::P_SWZ_MASK));
+                                    *dst = make_uint4(w[4 * jj], w[4 * jj + 1], w[4 * jj + 2], w[4 * jj + 3]);
+                                }
+                            }
+                        }
+                        if (rescale) {
+                            // O^T holds step 3 up to tile k-1: wait for it, then scale these columns in TMEM
+                            if (!waited_prev) {
+                                const int kp = k - 1;
+                                ok = ok && spin_phase<false>(bar(BR::PEMPTY + (kp % C::PB)), (kp / C::PB) & 1, abort_flag,
+                                                      status);
+                                tc_fence_after();
+                                waited_prev = true;
+                            }
+                            rescale_any = true;
+#pragma unroll
+                            for (int i = 0; i < C::PAIRS; ++i) {
+#pragma unroll
+                                for (int half = 0; half < 2; ++half) {
+                                    float v[16];
+                                    const uint32_t addr = tmem + lane_addr + C::O_COL + i * C::NP + half * NG + 16 * ch;
+                                    tmem_ld16(addr, v);
+                                    tmem_wait_ld();
+#pragma unroll
+                                    for (int n = 0; n < 16; ++n) v[n] *= alpha[n];
+                                    tmem_st16(addr, v);
+                                }
+                            }
+                        }
+                    }
+                    if (stop) break;
+                    if (rescale_any) tmem_wait_st();
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(BR::PFULL + pb));
+                }
+                if (stop) break;
+                // ---------------------------------------------------- epilogue: step 4 for this CTA's 256 columns
+                const int kl = k - 1;
+                ok = ok && spin_phase<false>(bar(BR::PEMPTY + (kl % C::PB)), (kl / C::PB) & 1, abort_flag, status);
+                tc_fence_after();
+#pragma unroll
+                for (int ch = 0; ch < C::CH; ++ch) {
+                    float v16[16];
+#pragma unroll
+                    for (int n = 0; n < 16; ++n) v16[n] = lpart[16 * ch + n];
+                    const float wsum = warp_colreduce16<false>(v16, lane);
+                    if ((lane & 1) == 0) redl[quad * NG + 16 * ch + col16(lane)] = wsum;
+                }
+                if (!named_bar_and(SMX, NSM, ok)) {  // also orders the redl writes before the reads
+                    stop = true;
+                    break;
+                }
+                const int nsplit = seq_info[4 * b + 2];
+                const int slot = seq_info[4 * b + 3] + (unit - seq_info[4 * b + 1]);
+#pragma unroll
+                for (int ch = 0; ch < C::CH; ++ch) {
+                    float inv_l[16], lse_n[16];
+#pragma unroll
+                    for (int n = 0; n < 16; ++n) {
+                        const int cn = 16 * ch + n;
+                        const float l = redl[cn] + redl[NG + cn] + redl[2 * NG + cn] + redl[3 * NG + cn];
+                        const bool empty = !(l > 0.f) || m[cn] == -INFINITY;
+                        inv_l[n] = empty ? 0.f : 1.f / l;
+                        lse_n[n] = empty ? -INFINITY : (m[cn] + __log2f(l)) * 0.69314718055994531f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < C::PAIRS; ++i) {
+                        float hi[16], lo[16];
+                        tmem_ld16(tmem + lane_addr + C::O_COL + i * C::NP + 16 * ch, hi);
+                        tmem_ld16(tmem + lane_addr + C::O_COL + i * C::NP + NG + 16 * ch, lo);
+                        tmem_wait_ld();
+                        const int d = 256 * (int)rank + 128 * i + row;
+#pragma unroll
+                        for (int n = 0; n < 16; ++n) {
+                            const int ng = grp * NG + 16 * ch + n;
+                            if (ng >= p.ncols) continue;
+                            const float val = (hi[n] + lo[n]) * inv_l[n];
+                            if (nsplit == 1)
+                                p.o[((int64_t)b * p.ncols + ng) * kDv + d] = __float2bfloat16_rn(val);
+                            else
+                                p.opart[((int64_t)slot * p.ncols + ng) * kDv + d] = val;
+                        }
+                    }
+                    if (rank == 0 && quad == 0 && lane < 16) {
+                        const int ng = grp * NG + 16 * ch + lane;
+                        float my = lse_n[0];
+#pragma unroll
+                        for (int n = 1; n < 16; ++n)
+                            if (lane == n) my = lse_n[n];
+                        if (ng < p.ncols) {
+                            if (nsplit == 1) p.lse[(int64_t)b * p.ncols + ng] = my;
+                            else p.lsepart[(int64_t)slot * p.ncols + ng] = my;
+                        }
+                    }
+                }
+                tc_fence_before();
+                ++seg;
+            }
+        }
+        if (stop || !ok) *abort_flag = 1;
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // no CTA leaves while its peer may still write into its shared memory
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace mla

@@ -13,7 +13,7 @@
 #include <string>
 
 #include "mla_decode.h"
-#include "etap_decode_kernel.cuh"
+#include "etap_pair_kernel.cuh"
 #include "plan_combine_kernels.cuh"
 #include "plan_core.h"
 
@@ -45,8 +45,9 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor map over a [rows, 576] row-major matrix; box = 64 columns x box_rows rows, 128B swizzle.
-int encode_rows_576(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows) {
+// 2-D bf16 tensor map over a [rows, 576] row-major matrix; box = box_cols columns x box_rows rows,
+// 128B swizzle for 64-column boxes, 64B swizzle for the 32-column rope boxes.
+int encode_rows_576(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows, uint32_t box_cols = 64) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) {
         g_last_cuda_error = "cuTensorMapEncodeTiled unavailable";
@@ -54,11 +55,12 @@ int encode_rows_576(CUtensorMap *map, const void *base, uint64_t rows, uint32_t 
     }
     cuuint64_t dims[2] = {(cuuint64_t)mla::kDqk, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)mla::kDqk * 2};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         g_last_cuda_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string((int)r);
         return MLA_ERR_CUDA;
@@ -74,7 +76,7 @@ int check_shape(int batch, int q_len, int num_heads, int num_sms) {
     return MLA_OK;
 }
 
-// Per-device one-time opt-in to the kernel's dynamic shared memory size.
+// Per-device one-time opt-in to the kernels' dynamic shared memory sizes.
 int ensure_smem_attr() {
     static std::mutex mu;
     static bool done[64] = {};
@@ -84,12 +86,34 @@ int ensure_smem_attr() {
     if (dev < 0 || dev >= 64) return MLA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(mu);
     if (!done[dev]) {
-        e = cudaFuncSetAttribute(mla::etap_decode_kernel<mla::Cfg16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)mla::Cfg16::SMEM_ALLOC);
+        e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)mla::PairCfg16::SMEM_ALLOC);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)mla::PairCfg64::SMEM_ALLOC);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         done[dev] = true;
     }
     return MLA_OK;
+}
+
+// One 2-CTA cluster per work unit and column group.
+template <class C>
+cudaError_t launch_pair(const CUtensorMap &tm_q, const CUtensorMap &tm_kv, const CUtensorMap &tm_qr,
+                        const CUtensorMap &tm_kvr, const mla::DecodeParams &p, int clusters, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.blockDim = dim3(192, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_ALLOC;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, mla::etap_pair_kernel<C>, tm_q, tm_kv, tm_qr, tm_kvr, p);
 }
 
 }  // namespace
@@ -217,10 +241,16 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
 
     st = ensure_smem_attr();
     if (st != MLA_OK) return st;
-    CUtensorMap tm_q, tm_kv;
-    st = encode_rows_576(&tm_q, q, (uint64_t)batch * ncols, mla::Cfg16::NG);
+    CUtensorMap tm_q, tm_kv, tm_qr, tm_kvr;
+    const int ng = mla::group_cols(ncols);
+    const uint64_t kv_total_rows = paged ? (uint64_t)kv_rows : (uint64_t)batch * kv_rows;
+    st = encode_rows_576(&tm_q, q, (uint64_t)batch * ncols, (uint32_t)ng);
     if (st != MLA_OK) return st;
-    st = encode_rows_576(&tm_kv, kv, paged ? (uint64_t)kv_rows : (uint64_t)batch * kv_rows, 64);
+    st = encode_rows_576(&tm_kv, kv, kv_total_rows, 64);
+    if (st != MLA_OK) return st;
+    st = encode_rows_576(&tm_qr, q, (uint64_t)batch * ncols, (uint32_t)ng, 32);
+    if (st != MLA_OK) return st;
+    st = encode_rows_576(&tm_kvr, kv, kv_total_rows, 64, 32);
     if (st != MLA_OK) return st;
 
     char *ws = reinterpret_cast<char *>(workspace);
@@ -248,9 +278,11 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
     p.seq_info_off = (int)(lay.seq_info / 4);
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    mla::etap_decode_kernel<mla::Cfg16><<<lay.ctas * lay.groups, 192, mla::Cfg16::SMEM_ALLOC, s>>>(tm_q, tm_kv, p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "etap_decode_kernel launch");
+    cudaError_t e = ng == 16 ? launch_pair<mla::PairCfg16>(tm_q, tm_kv, tm_qr, tm_kvr, p, lay.ctas * lay.groups, s)
+                             : launch_pair<mla::PairCfg64>(tm_q, tm_kv, tm_qr, tm_kvr, p, lay.ctas * lay.groups, s);
+    if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
     if (!(flags & MLA_FLAG_SKIP_COMBINE))
         return mla_combine(workspace, batch, q_len, num_heads, num_sms, o, lse, stream);
     return MLA_OK;

@@ -21,7 +21,6 @@
 namespace mla {
 
 constexpr int kTileRows = 128;   // KV rows per tile = UMMA M of S^T = K Q^T
-constexpr int kColGroup = 16;    // query columns (heads x tokens) per CTA = UMMA N of S^T
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kPage = 64;
@@ -39,9 +38,13 @@ enum : int {
     kHdrWords = 64
 };
 
-MLA_HD int num_groups(int ncols) { return (ncols + kColGroup - 1) / kColGroup; }
+// Query columns (heads x tokens) per cluster = UMMA N of S^T: one group of 16
+// when they fit, otherwise groups of 64.
+MLA_HD int group_cols(int ncols) { return ncols <= 16 ? 16 : 64; }
+MLA_HD int num_groups(int ncols) { return (ncols + group_cols(ncols) - 1) / group_cols(ncols); }
+// Work units per column group: one per pair of SMs (a 2-CTA cluster).
 MLA_HD int num_ctas(int num_sms, int groups) {
-    int c = num_sms / groups;
+    int c = num_sms / 2 / groups;
     return c < 1 ? 1 : c;
 }
 MLA_HD int tiles_of(int L) { return L <= 0 ? 0 : (L + kTileRows - 1) / kTileRows; }
@@ -60,7 +63,7 @@ MLA_HD int cta_of(int64_t total, int used, int64_t f) { return (int)(((f + 1) * 
 MLA_HD size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct WsLayout {
-    size_t cta_ranges;  // int32 [ctas][2]
+    size_t cta_ranges;  // int32 [ctas][2] (one range per work unit = SM pair)
     size_t tile_off;    // int32 [batch + 1]
     size_t seq_info;    // int32 [batch][4]: tiles, first CTA, splits, slot offset
     size_t opart;       // fp32  [slots][ncols][512]

@@ -21,8 +21,9 @@ def test_schedule_invariants(seed, n_sms, h, q):
     lens = rng.integers(0, 70000, B)
     lens[rng.random(B) < 0.2] = 0
     ranges, info, ctas, groups = m.mla_decode_plan_host(lens, q, h, n_sms)
-    assert groups == (q * h + 15) // 16
-    assert ctas == max(1, n_sms // groups)
+    ncols = q * h
+    assert groups == (1 if ncols <= 16 else (ncols + 63) // 64)
+    assert ctas == max(1, n_sms // 2 // groups)  # one work unit per SM pair
     T = sum(tiles(int(L)) for L in lens)
     # the CTA ranges tile [0, T) in order; the working CTAs come first, each with
     # at least one tile, sizes within 1 of each other; idle CTAs (only when T < ctas) come last
@@ -68,7 +69,7 @@ def test_fewer_tiles_than_ctas(lens, n_sms):
 
 def test_headline_shape_balance():
     ranges, info, ctas, groups = m.mla_decode_plan_host([65536] * 16, 1, 16, 148)
-    assert ctas == 148 and groups == 1
+    assert ctas == 74 and groups == 1
     sizes = ranges[:, 1] - ranges[:, 0]
-    assert sizes.min() == 55 and sizes.max() == 56
-    assert np.all(info[:, 2] >= 9)
+    assert sizes.min() == 110 and sizes.max() == 111
+    assert np.all(info[:, 2] >= 5)
