@@ -41,7 +41,8 @@ METRIC = "MLA decode TB/s & TFLOPS (B=16,h=16,64K KV) as % of B200 roofline"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-KERNEL_SOURCES = ["mla_decode_attention_etap_b200/csrc/etap_decode_kernel.cuh",
+KERNEL_SOURCES = ["mla_decode_attention_etap_b200/csrc/etap_pair_kernel.cuh",
+                  "mla_decode_attention_etap_b200/csrc/etap_common.cuh",
                   "mla_decode_attention_etap_b200/csrc/ptx_sm100.cuh",
                   "mla_decode_attention_etap_b200/csrc/plan_core.h"]
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "etap_decode_kernel_ncu.md")
@@ -381,7 +382,7 @@ def run_ours(args):
             roof = {"bound": "tensor", "achieved": ach, "peak": tc_tflops, "unit": "TFLOP/s", "frac": ach / tc_tflops}
         roof["traffic"] = profiled_traffic(wname)
         roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
-        roof["kernel"] = "etap_decode_kernel"
+        roof["kernel"] = "etap_pair_kernel"
         roof["kernel_ms"] = kern_s * 1e3
         roof["tflops"] = flops / kern_s / 1e12
         roof["algorithmic_bytes_per_launch"] = kv_bytes
