@@ -47,6 +47,7 @@ struct PairCfg {
     static constexpr int PAIRS = 2;                                    // V pairs of a tile in one CTA
     static constexpr int EARLY = (NV - PAIRS) < PAIRS ? (NV - PAIRS) : PAIRS;  // pairs of tile k+1 free of tile k
     static constexpr int XS = 2;                                       // exchange slots
+    static constexpr int PREFETCH = 2;                                 // tiles the L2 prefetch runs ahead of the loads
     static constexpr uint32_t CHUNK = 16384;                           // 128 rows x 64 bf16, 128B swizzle
     static constexpr uint32_t HALF = 8192;                             // 64 rows of a chunk = one TMA box
     static constexpr uint32_t V_SLOT = 2 * CHUNK;
@@ -208,6 +209,34 @@ __global__ void __launch_bounds__(192, 1)
         for (int i = 0; i < C::NR; ++i) arms_r[i] = 0;
         int arms_q = 0, tail_uses = 0;
         bool ok = true;
+        // L2 prefetch of this CTA's columns of a future tile, so that the load that
+        // refills a freed slot hits L2 instead of waiting on HBM.
+        auto prefetch_tile = [&](int pb_, int pt_) {
+            int Lp = p.seqlens[pb_];
+            if ((int64_t)Lp > l_cap) Lp = (int)l_cap;
+            const int r0 = pt_ * kTileRows;
+            for (int hh = 0; hh < 2; ++hh) {
+                if (Lp - r0 <= 64 * hh) break;
+                int yp;
+                if (p.paged) {
+                    const int blk = p.block_table[(int64_t)pb_ * p.max_blocks + (r0 >> 6) + hh];
+                    if (blk < 0 || (int64_t)blk * kPage >= p.kv_rows) continue;
+                    yp = blk * kPage;
+                } else {
+                    yp = (int)((int64_t)pb_ * p.kv_rows + r0 + 64 * hh);
+                }
+                for (int c = 0; c < 4; ++c) tma_prefetch_l2_2d(&tm_kv, (4 * (int)rank + c) * 64, yp);
+                tma_prefetch_l2_2d(&tm_kvr, rope_x, yp);
+            }
+        };
+        TileCursor ahead;
+        if (fb < fe && lane == 0) {
+            ahead.init(tile_off, p.batch, fb, fe);
+            for (int d = 0; d < C::PREFETCH && ahead.valid; ++d) {
+                prefetch_tile(ahead.b, ahead.t);
+                ahead.advance(tile_off);
+            }
+        }
         if (fb < fe) {
             SegIter it;
             it.init(tile_off, p.batch, fb, fe);
@@ -231,6 +260,10 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 ++arms_q;
                 for (int t = t0; t < t1 && ok; ++t, ++k) {
+                    if (lane == 0 && ahead.valid) {
+                        prefetch_tile(ahead.b, ahead.t);
+                        ahead.advance(tile_off);
+                    }
                     const int row0 = t * kTileRows;
                     int valid = L - row0;
                     valid = valid < 0 ? 0 : (valid > kTileRows ? kTileRows : valid);
