@@ -67,7 +67,11 @@ enum {
 
 /* Flags for mla_decode_fwd. */
 enum {
-    MLA_FLAG_SKIP_COMBINE = 1 /* leave split partials in the workspace; call mla_combine yourself */
+    MLA_FLAG_SKIP_COMBINE = 1, /* leave split partials in the workspace; call mla_combine yourself */
+    /* Test hook for failure detection: the kernel never loads Q, so its bounded waits run out
+     * (after 100 ms instead of the normal 4 s); the call still returns MLA_OK and
+     * mla_decode_read_status then reports MLA_ERR_TIMEOUT. Outputs are undefined. */
+    MLA_FLAG_TEST_EXPIRE_WAITS = 0x40000000
 };
 
 /*

@@ -21,6 +21,7 @@ D_QK = 576
 D_V = 512
 PAGE_SIZE = 64
 FLAG_SKIP_COMBINE = 1
+FLAG_TEST_EXPIRE_WAITS = 0x40000000
 
 STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3: "MLA_ERR_ALIGNMENT",
           -4: "MLA_ERR_WORKSPACE", -5: "MLA_ERR_CUDA", -6: "MLA_ERR_TIMEOUT", -7: "MLA_ERR_BLOCK_TABLE"}

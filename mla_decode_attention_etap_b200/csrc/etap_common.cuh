@@ -14,9 +14,18 @@ namespace mla {
 constexpr int kStatusTimeout = -6;      // MLA_ERR_TIMEOUT
 constexpr int kStatusBlockTable = -7;   // MLA_ERR_BLOCK_TABLE
 constexpr int kStatusInvalid = -1;      // MLA_ERR_INVALID_ARG
-constexpr uint64_t kWaitLimitNs = 4000000000ull;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;     // default bound of every wait
+constexpr uint64_t kTestWaitLimitNs = 100000000ull;  // bound used by the expired-wait test hook
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p = 2^(x - m) stays <= 256
+
+// Per-CTA wait control in shared memory: the abort flag every role polls and
+// the bound after which a wait gives up.
+struct WaitCtl {
+    int abort;
+    int pad;
+    unsigned long long limit_ns;
+};
 
 struct DecodeParams {
     const int32_t *seqlens;
@@ -29,21 +38,23 @@ struct DecodeParams {
     int64_t kv_rows;  // contiguous: rows per sequence; paged: total rows of the pool
     int batch, q_len, num_heads, ncols, ctas, groups, max_blocks, paged, causal;
     float scale_log2;  // softmax_scale * log2(e)
+    unsigned long long wait_limit_ns;
+    int withhold_q;    // test hook: never load Q, so that the bounded waits expire
     int cta_ranges_off, tile_off_off, seq_info_off;  // int32 offsets into ws
 };
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA abort
 // flag) when the wait ran past kWaitLimitNs, or when another role aborted.
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile WaitCtl *wc,
                                            int32_t *status) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t spin = 1;; ++spin) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((spin & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
-                *abort_flag = 1;
+            if (wc->abort) return false;
+            if (global_timer_ns() - t0 > wc->limit_ns) {
+                wc->abort = 1;
                 atomicCAS(status, 0, kStatusTimeout);
                 return false;
             }
@@ -163,7 +174,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // resumes the moment the phase completes (a suspended try_wait can wake late,
 // and the slowest of the 128 threads sets the pace of the next named barrier).
 template <bool CLUSTER>
-__device__ __forceinline__ bool spin_phase(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+__device__ __forceinline__ bool spin_phase(uint32_t bar, uint32_t parity, volatile WaitCtl *wc,
                                            int32_t *status) {
     auto probe = [&]() { return CLUSTER ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity); };
     if (probe()) return true;
@@ -171,9 +182,9 @@ __device__ __forceinline__ bool spin_phase(uint32_t bar, uint32_t parity, volati
     for (uint32_t spin = 1;; ++spin) {
         if (probe()) return true;
         if ((spin & 255u) == 0) {
-            if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
-                *abort_flag = 1;
+            if (wc->abort) return false;
+            if (global_timer_ns() - t0 > wc->limit_ns) {
+                wc->abort = 1;
                 atomicCAS(status, 0, kStatusTimeout);
                 return false;
             }
@@ -182,16 +193,16 @@ __device__ __forceinline__ bool spin_phase(uint32_t bar, uint32_t parity, volati
 }
 
 // Bounded wait on a phase completed by the peer CTA of the cluster (acquire at cluster scope).
-__device__ __forceinline__ bool wait_phase_cluster(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+__device__ __forceinline__ bool wait_phase_cluster(uint32_t bar, uint32_t parity, volatile WaitCtl *wc,
                                                    int32_t *status) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t spin = 1;; ++spin) {
         if (mbar_try_wait_cluster(bar, parity)) return true;
         if ((spin & 63u) == 0) {
-            if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
-                *abort_flag = 1;
+            if (wc->abort) return false;
+            if (global_timer_ns() - t0 > wc->limit_ns) {
+                wc->abort = 1;
                 atomicCAS(status, 0, kStatusTimeout);
                 return false;
             }

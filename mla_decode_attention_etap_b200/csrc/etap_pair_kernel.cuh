@@ -46,7 +46,7 @@ struct PairCfg {
     static constexpr int NV = NV_, NR = NR_, PB = PB_;
     static constexpr int PAIRS = 2;                                    // V pairs of a tile in one CTA
     static constexpr int EARLY = (NV - PAIRS) < PAIRS ? (NV - PAIRS) : PAIRS;  // pairs of tile k+1 free of tile k
-    static constexpr int XS = 2;                                       // exchange slots
+    static constexpr int XS = CH > 2 ? CH : 2;                         // exchange slots (8 KB each)
     static constexpr int PREFETCH = 2;                                 // tiles the L2 prefetch runs ahead of the loads
     static constexpr uint32_t CHUNK = 16384;                           // 128 rows x 64 bf16, 128B swizzle
     static constexpr uint32_t HALF = 8192;                             // 64 rows of a chunk = one TMA box
@@ -107,7 +107,8 @@ struct PairBars {
     static constexpr int RED = FINAL + 1;
     static constexpr int REDL = RED + 1;
     static constexpr int XFULL = REDL + 1;
-    static constexpr int COUNT = XFULL + C::XS;
+    static constexpr int XFREE = XFULL + C::XS;  // used when CH > 1: the peer consumed our last tile
+    static constexpr int COUNT = XFREE + 1;
 };
 static_assert(PairBars<PairCfg16>::COUNT * 8 <= 512 && PairBars<PairCfg64>::COUNT * 8 <= 512, "barrier area");
 
@@ -143,7 +144,7 @@ __global__ void __launch_bounds__(192, 1)
     const bool plan_ok = p.ws[kHdrCtas] == p.ctas && p.ws[kHdrGroups] == p.groups && p.ws[kHdrBatch] == p.batch;
 
     auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * (uint32_t)i; };
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    volatile WaitCtl *wc = reinterpret_cast<volatile WaitCtl *>(smem + C::OFF_MISC + 16);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
 
     if (threadIdx.x == 0) {
@@ -170,7 +171,9 @@ __global__ void __launch_bounds__(192, 1)
         mbar_init(bar(BR::RED), 4);
         mbar_init(bar(BR::REDL), 4);
         for (int i = 0; i < C::XS; ++i) mbar_init(bar(BR::XFULL + i), 1);
-        *abort_flag = 0;
+        mbar_init(bar(BR::XFREE), 4);
+        wc->abort = 0;
+        wc->limit_ns = p.wait_limit_ns;
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
@@ -248,9 +251,9 @@ __global__ void __launch_bounds__(192, 1)
                     L = (int)l_cap;
                 }
                 if (L < 0) L = 0;
-                if (seg > 0) ok = wait_phase(bar(BR::QEMPTY), (seg - 1) & 1, abort_flag, status);
+                if (seg > 0) ok = wait_phase(bar(BR::QEMPTY), (seg - 1) & 1, wc, status);
                 if (!ok) break;
-                if (lane == 0) {
+                if (lane == 0 && !p.withhold_q) {
                     mbar_arrive_expect_tx(bar(BR::QFULL), 4 * C::Q_CHUNK + C::Q_ROPE);
                     const int qrow = b * p.ncols + grp * NG;
                     for (int j = 0; j < 4; ++j)
@@ -258,7 +261,7 @@ __global__ void __launch_bounds__(192, 1)
                                     qrow);
                     tma_load_2d(sbase + C::OFF_QR, &tm_qr, bar(BR::QFULL), rope_x, qrow);
                 }
-                ++arms_q;
+                if (!p.withhold_q) ++arms_q;
                 for (int t = t0; t < t1 && ok; ++t, ++k) {
                     if (lane == 0 && ahead.valid) {
                         prefetch_tile(ahead.b, ahead.t);
@@ -292,7 +295,7 @@ __global__ void __launch_bounds__(192, 1)
                     {
                         // this CTA's 32 rope columns: rows past the end are masked in S^T, no zeroing needed
                         const int rs = k % C::NR;
-                        ok = wait_phase(bar(BR::REMPTY + rs), ((k / C::NR) & 1) ^ 1, abort_flag, status);
+                        ok = wait_phase(bar(BR::REMPTY + rs), ((k / C::NR) & 1) ^ 1, wc, status);
                         if (!ok) break;
                         if (lane == 0) {
                             mbar_arrive_expect_tx(bar(BR::RFULL + rs), nload * C::R_HALF);
@@ -307,7 +310,7 @@ __global__ void __launch_bounds__(192, 1)
                         const int g2 = C::PAIRS * k + i;
                         const int vs = g2 % C::NV;
                         const int c0 = 4 * (int)rank + 2 * i;  // latent chunks c0, c0+1 of this CTA's half
-                        ok = wait_phase(bar(BR::VEMPTY + vs), ((g2 / C::NV) & 1) ^ 1, abort_flag, status);
+                        ok = wait_phase(bar(BR::VEMPTY + vs), ((g2 / C::NV) & 1) ^ 1, wc, status);
                         if (!ok) break;
                         const uint32_t dst = sbase + C::OFF_V + vs * C::V_SLOT;
                         if (!tail) {
@@ -332,7 +335,7 @@ __global__ void __launch_bounds__(192, 1)
                                                 tma_load_2d(dst + hc * C::CHUNK + hh * C::HALF, &tm_kv, bar(BR::TAIL),
                                                             (c0 + hc) * 64, y[hh]);
                                 }
-                                ok = wait_phase(bar(BR::TAIL), tail_uses & 1, abort_flag, status);
+                                ok = wait_phase(bar(BR::TAIL), tail_uses & 1, wc, status);
                                 ++tail_uses;
                                 if (!ok) break;
                             }
@@ -453,10 +456,10 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 if (progressed) {
                     t_last = global_timer_ns();
-                } else if (*abort_flag) {
+                } else if (wc->abort) {
                     break;
-                } else if (global_timer_ns() - t_last > kWaitLimitNs) {
-                    *abort_flag = 1;
+                } else if (global_timer_ns() - t_last > wc->limit_ns) {
+                    wc->abort = 1;
                     atomicCAS(status, 0, kStatusTimeout);
                     break;
                 }
@@ -478,7 +481,27 @@ __global__ void __launch_bounds__(192, 1)
         float *redl = reinterpret_cast<float *>(smem + C::OFF_REDL);  // [4][NG]
         const uint32_t x_remote = map_to_rank(sbase + C::OFF_X, peer);
         const uint32_t xfull_remote = map_to_rank(bar(BR::XFULL), peer);
+        const uint32_t xfree_remote = map_to_rank(bar(BR::XFREE), peer);
+        const int k_total = (int)(fe - fb);
         bool ok = true, stop = false;
+        // CH > 1: whole-tile exchange, one tile ahead.  Our partial S^T of tile kk goes to the
+        // peer's slots 0..CH-1 once the peer has combined tile kk-1 (XFREE).
+        auto send_tile = [&](int kk) {
+            ok = ok && spin_phase<false>(bar(BR::SFULL + (kk & 1)), (kk >> 1) & 1, wc, status);
+            tc_fence_after();
+            ok = ok && spin_phase<true>(bar(BR::XFREE), (kk & 1) ^ 1, wc, status);
+#pragma unroll
+            for (int ch = 0; ch < C::CH; ++ch) {
+                float xs16[16];
+                tmem_ld16(tmem + lane_addr + C::S_COL + (kk & 1) * NG + 16 * ch, xs16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 4 && ok; ++j)
+                    st_async_v4(x_remote + ch * C::X_SLOT + swz_off(row, j, 64, 3), __float_as_uint(xs16[4 * j]),
+                                __float_as_uint(xs16[4 * j + 1]), __float_as_uint(xs16[4 * j + 2]),
+                                __float_as_uint(xs16[4 * j + 3]), xfull_remote);
+            }
+        };
         if (fb < fe) {
             SegIter it;
             it.init(tile_off, p.batch, fb, fe);
@@ -496,12 +519,45 @@ __global__ void __launch_bounds__(192, 1)
                 for (int t = t0; t < t1 && !stop; ++t, ++k) {
                     const bool first = (t == t0);
                     const int pb = k % C::PB;
-                    ok = ok && spin_phase<false>(bar(BR::SFULL + (k & 1)), (k >> 1) & 1, abort_flag, status);
+                    ok = ok && spin_phase<false>(bar(BR::SFULL + (k & 1)), (k >> 1) & 1, wc, status);
                     tc_fence_after();
                     const int rg = t * kTileRows + row;
                     // every row of the tile visible to every column: no per-column mask needed
                     const bool full_tile = (t + 1) * kTileRows <= (p.causal ? L - p.q_len + 1 : L);
-                    bool waited_prev = false, rescale_any = false;
+                    bool waited_prev = false, rescale_any = false, sent_next = false;
+                    if constexpr (C::CH > 1) {
+                        // (a) add the peer's partial S^T of tile k into ours, in TMEM, and free its slots;
+                        // (b) send our partial of tile k+1 so it travels while tile k's softmax runs.
+                        if (k == 0) send_tile(0);
+                        if (row == 0) mbar_arrive_expect_tx(bar(BR::XFULL), C::CH * C::X_SLOT);
+                        ok = ok && spin_phase<true>(bar(BR::XFULL), k & 1, wc, status);
+#pragma unroll
+                        for (int ch = 0; ch < C::CH; ++ch) {
+                            float xo[16];
+                            const uint32_t taddr = tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch;
+                            tmem_ld16(taddr, xo);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float4 v = *reinterpret_cast<const float4 *>(smem + C::OFF_X + ch * C::X_SLOT +
+                                                                                   swz_off(row, j, 64, 3));
+                                xo[4 * j] += v.x;
+                                xo[4 * j + 1] += v.y;
+                                xo[4 * j + 2] += v.z;
+                                xo[4 * j + 3] += v.w;
+                            }
+                            tmem_st16(taddr, xo);
+                        }
+                        tmem_wait_st();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_remote(xfree_remote);
+                        // Send now only if S^T of tile k+1 is already there: with few V slots its
+                        // scores can depend on step 3 of tile k, i.e. on this tile's softmax.
+                        if (k + 1 < k_total && mbar_test_wait(bar(BR::SFULL + ((k + 1) & 1)), ((k + 1) >> 1) & 1)) {
+                            send_tile(k + 1);
+                            sent_next = true;
+                        }
+                    }
 #pragma unroll
                     for (int ch = 0; ch < C::CH; ++ch) {
                         float x[16];
@@ -512,6 +568,7 @@ __global__ void __launch_bounds__(192, 1)
                             __syncwarp();
                             if (lane == 0) mbar_arrive(bar(BR::SEMPTY + (k & 1)));
                         }
+                        if constexpr (C::CH == 1) {
                         // ---- exchange of the partial scores with the peer CTA.  Slot xs is free for
                         // exchange e without a handshake: the peer overwrites it (exchange e + XS) only
                         // after receiving our exchange e + XS - 1, which we send after consuming e.
@@ -519,12 +576,12 @@ __global__ void __launch_bounds__(192, 1)
                         const int xs = e % C::XS, xu = e / C::XS;
                         ++e;
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
+                        for (int j = 0; j < 4 && ok; ++j)
                             st_async_v4(x_remote + xs * C::X_SLOT + swz_off(row, j, 64, 3), __float_as_uint(x[4 * j]),
                                         __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
                                         __float_as_uint(x[4 * j + 3]), xfull_remote + 8u * xs);
                         if (row == 0) mbar_arrive_expect_tx(bar(BR::XFULL + xs), C::X_SLOT);
-                        ok = ok && spin_phase<true>(bar(BR::XFULL + xs), xu & 1, abort_flag, status);
+                        ok = ok && spin_phase<true>(bar(BR::XFULL + xs), xu & 1, wc, status);
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
                             const float4 v = *reinterpret_cast<const float4 *>(smem + C::OFF_X + xs * C::X_SLOT +
@@ -534,6 +591,7 @@ __global__ void __launch_bounds__(192, 1)
                             x[4 * j + 2] += v.z;
                             x[4 * j + 3] += v.w;
                         }
+                        }  // CH == 1 exchange
                         // ---- scale + mask
                         if (full_tile) {
 #pragma unroll
@@ -602,7 +660,7 @@ __global__ void __launch_bounds__(192, 1)
                         }
                         // ---- P^T row chunk -> shared memory: bf16 hi into columns [16ch, 16ch+16), lo into NG + that
                         if (ch == 0)
-                            ok = ok && spin_phase<false>(bar(BR::PEMPTY + pb), ((k / C::PB) & 1) ^ 1, abort_flag, status);
+                            ok = ok && spin_phase<false>(bar(BR::PEMPTY + pb), ((k / C::PB) & 1) ^ 1, wc, status);
                         {
                             uint32_t hi[8], lo[8];
 #pragma unroll
@@ -632,7 +690,7 @@ __global__ void __launch_bounds__(192, 1)
                             // O^T holds step 3 up to tile k-1: wait for it, then scale these columns in TMEM
                             if (!waited_prev) {
                                 const int kp = k - 1;
-                                ok = ok && spin_phase<false>(bar(BR::PEMPTY + (kp % C::PB)), (kp / C::PB) & 1, abort_flag,
+                                ok = ok && spin_phase<false>(bar(BR::PEMPTY + (kp % C::PB)), (kp / C::PB) & 1, wc,
                                                       status);
                                 tc_fence_after();
                                 waited_prev = true;
@@ -659,11 +717,14 @@ __global__ void __launch_bounds__(192, 1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(BR::PFULL + pb));
+                    if constexpr (C::CH > 1) {
+                        if (k + 1 < k_total && !sent_next) send_tile(k + 1);
+                    }
                 }
                 if (stop) break;
                 // ---------------------------------------------------- epilogue: step 4 for this CTA's 256 columns
                 const int kl = k - 1;
-                ok = ok && spin_phase<false>(bar(BR::PEMPTY + (kl % C::PB)), (kl / C::PB) & 1, abort_flag, status);
+                ok = ok && spin_phase<false>(bar(BR::PEMPTY + (kl % C::PB)), (kl / C::PB) & 1, wc, status);
                 tc_fence_after();
 #pragma unroll
                 for (int ch = 0; ch < C::CH; ++ch) {
@@ -724,13 +785,21 @@ __global__ void __launch_bounds__(192, 1)
                 ++seg;
             }
         }
-        if (stop || !ok) *abort_flag = 1;
+        if (stop || !ok) wc->abort = 1;
         __syncwarp();
     }
 
     tc_fence_before();
     __syncthreads();
     cluster_sync();  // no CTA leaves while its peer may still write into its shared memory
+    if (wc->abort) {
+        // After an abort a peer's last st.async may not have been waited for: let it land
+        // before either CTA leaves (no thread sends after the barrier above).
+        const uint64_t t_q = global_timer_ns();
+        while (global_timer_ns() - t_q < 20000ull) {
+        }
+    }
+    cluster_sync();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
 }

@@ -222,7 +222,7 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
     if (!q || !kv || !seqlens || !o || !lse || !workspace) return MLA_ERR_INVALID_ARG;
     if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
-    if ((flags & ~(unsigned)MLA_FLAG_SKIP_COMBINE) != 0) return MLA_ERR_INVALID_ARG;
+    if ((flags & ~(unsigned)(MLA_FLAG_SKIP_COMBINE | MLA_FLAG_TEST_EXPIRE_WAITS)) != 0) return MLA_ERR_INVALID_ARG;
     if (kv_rows < 1) return MLA_ERR_INVALID_ARG;
     const bool paged = block_table != nullptr;
     if (paged) {
@@ -273,6 +273,8 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
     p.paged = paged ? 1 : 0;
     p.causal = causal;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
+    p.wait_limit_ns = (flags & MLA_FLAG_TEST_EXPIRE_WAITS) ? mla::kTestWaitLimitNs : mla::kWaitLimitNs;
+    p.withhold_q = (flags & MLA_FLAG_TEST_EXPIRE_WAITS) ? 1 : 0;
     p.cta_ranges_off = (int)(lay.cta_ranges / 4);
     p.tile_off_off = (int)(lay.tile_off / 4);
     p.seq_info_off = (int)(lay.seq_info / 4);

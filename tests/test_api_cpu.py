@@ -70,7 +70,7 @@ def fwd(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(q=0), -1), (dict(kv=0), -1), (dict(o=0), -1), (dict(lse=0), -1), (dict(ws=0), -1),
     (dict(scale=0.0), -1), (dict(scale=-1.0), -1), (dict(scale=float("inf")), -1), (dict(scale=float("nan")), -1),
-    (dict(causal=2), -1), (dict(flags=8), -1), (dict(batch=0), -1), (dict(q_len=0), -1),
+    (dict(causal=2), -1), (dict(flags=8), -1), (dict(flags=0x20000000), -1), (dict(batch=0), -1), (dict(q_len=0), -1),
     (dict(num_heads=2048), -2), (dict(kv_rows=0), -1),
     (dict(q=A + 8), -3), (dict(kv=A + 2), -3), (dict(o=A + 4), -3), (dict(lse=A + 2), -3), (dict(ws=A + 16), -3),
     (dict(ws_bytes=100), -4),

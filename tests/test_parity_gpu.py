@@ -191,3 +191,18 @@ def test_full_b32_h128_paged_sampled():
 def test_full_b16_h16_q4_causal_sampled():
     w = W.workload_b16_h16_q4_causal(seed=0, device="cuda")
     _full(w, [0, 9])
+
+
+def test_bounded_waits_report_timeout_and_context_survives():
+    """Failure detection without a GPU fault: with Q withheld the kernel's bounded waits
+    run out (100 ms), it records MLA_ERR_TIMEOUT and returns; the next call is correct."""
+    from mla_decode_attention_etap_b200 import FLAG_TEST_EXPIRE_WAITS
+    w = W.make_workload(2, 16, [3000, 700], seed=15)
+    _, _, st, dec = run_cuda(w, flags=FLAG_TEST_EXPIRE_WAITS, poison=False)
+    assert st == -6  # MLA_ERR_TIMEOUT
+    o, lse, st2, _ = run_cuda(w, decoder=dec)
+    assert st2 == 0
+    assert_parity(o, lse, *run_oracle(w), what="after an expired wait")
+    w2 = W.make_workload(1, 128, [500], seed=16)
+    _, _, st3, _ = run_cuda(w2, flags=FLAG_TEST_EXPIRE_WAITS, poison=False)
+    assert st3 == -6
