@@ -45,7 +45,7 @@ KERNEL_SOURCES = ["mla_decode_attention_etap_b200/csrc/etap_pair_kernel.cuh",
                   "mla_decode_attention_etap_b200/csrc/etap_common.cuh",
                   "mla_decode_attention_etap_b200/csrc/ptx_sm100.cuh",
                   "mla_decode_attention_etap_b200/csrc/plan_core.h"]
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "etap_decode_kernel_ncu.md")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "etap_pair_kernel_ncu.md")
 
 WORKLOADS = {
     "b16_h16_64k": dict(batch=16, heads=16, seqlen=65536),
