@@ -387,45 +387,11 @@ __global__ void __launch_bounds__(192, 1)
             qc.init(tile_off, p.batch, fb, fe);
             pc.init(tile_off, p.batch, fb, fe);
             int kq = 0, kp = 0, seg_q = 0;
+            int qstage = 0;  // scores of tile kq: 0 = rope columns next, 1 + i = V pair i next
             uint64_t t_last = global_timer_ns();
             while (pc.valid) {
                 bool progressed = false;
-                if (qc.valid) {
-                    const int rs = kq % C::NR;
-                    bool ready = mbar_test_wait(bar(BR::SEMPTY + (kq & 1)), ((kq >> 1) & 1) ^ 1);
-                    if (ready && qc.first()) ready = mbar_test_wait(bar(BR::QFULL), seg_q & 1);
-                    if (ready) ready = mbar_test_wait(bar(BR::RFULL + rs), (kq / C::NR) & 1);
-                    for (int i = 0; i < C::PAIRS && ready; ++i) {
-                        const int g2 = C::PAIRS * kq + i;
-                        ready = mbar_test_wait(bar(BR::VFULL + g2 % C::NV), (g2 / C::NV) & 1);
-                    }
-                    if (ready) {
-                        tc_fence_after();
-                        const uint32_t d_s = tmem + C::S_COL + (kq & 1) * NG;
-                        // 32 rope columns (K-major, 64-byte rows): two K-steps; the first (re)initialises S^T
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const uint64_t a = smem_desc(sbase + C::OFF_R + rs * C::R_SLOT + 32u * j, 16, 512, kSwizzle64B);
-                            const uint64_t bq = smem_desc(sbase + C::OFF_QR + 32u * j, 16, 512, kSwizzle64B);
-                            umma_bf16(d_s, a, bq, C::IDESC_QK, j == 0 ? 0u : 1u);
-                        }
-                        umma_commit(bar(BR::REMPTY + rs));
-                        for (int i = 0; i < C::PAIRS; ++i) {
-                            const int g2 = C::PAIRS * kq + i;
-                            const uint32_t slot = sbase + C::OFF_V + (g2 % C::NV) * C::V_SLOT;
-                            qk_chunk(d_s, slot, 2 * i, false);
-                            qk_chunk(d_s, slot + C::CHUNK, 2 * i + 1, false);
-                        }
-                        umma_commit(bar(BR::SFULL + (kq & 1)));
-                        if (qc.last()) {
-                            umma_commit(bar(BR::QEMPTY));
-                            ++seg_q;
-                        }
-                        qc.advance(tile_off);
-                        ++kq;
-                        progressed = true;
-                    }
-                }
+                // step 3 first when its P^T is ready: it frees V slots for later tiles
                 if (kp < kq) {
                     const int pb = kp % C::PB;
                     if (mbar_test_wait(bar(BR::PFULL + pb), (kp / C::PB) & 1)) {
@@ -452,6 +418,51 @@ __global__ void __launch_bounds__(192, 1)
                         pc.advance(tile_off);
                         ++kp;
                         progressed = true;
+                    }
+                }
+                // step 1 in stages, each as soon as its operands have landed
+                if (qc.valid) {
+                    const uint32_t d_s = tmem + C::S_COL + (kq & 1) * NG;
+                    if (qstage == 0) {
+                        const int rs = kq % C::NR;
+                        bool ready = mbar_test_wait(bar(BR::SEMPTY + (kq & 1)), ((kq >> 1) & 1) ^ 1);
+                        if (ready && qc.first()) ready = mbar_test_wait(bar(BR::QFULL), seg_q & 1);
+                        if (ready) ready = mbar_test_wait(bar(BR::RFULL + rs), (kq / C::NR) & 1);
+                        if (ready) {
+                            tc_fence_after();
+                            // 32 rope columns (K-major, 64-byte rows): two K-steps; the first (re)initialises S^T
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                const uint64_t a =
+                                    smem_desc(sbase + C::OFF_R + rs * C::R_SLOT + 32u * j, 16, 512, kSwizzle64B);
+                                const uint64_t bq = smem_desc(sbase + C::OFF_QR + 32u * j, 16, 512, kSwizzle64B);
+                                umma_bf16(d_s, a, bq, C::IDESC_QK, j == 0 ? 0u : 1u);
+                            }
+                            umma_commit(bar(BR::REMPTY + rs));
+                            qstage = 1;
+                            progressed = true;
+                        }
+                    }
+                    if (qstage >= 1) {
+                        const int i = qstage - 1;
+                        const int g2 = C::PAIRS * kq + i;
+                        if (mbar_test_wait(bar(BR::VFULL + g2 % C::NV), (g2 / C::NV) & 1)) {
+                            tc_fence_after();
+                            const uint32_t slot = sbase + C::OFF_V + (g2 % C::NV) * C::V_SLOT;
+                            qk_chunk(d_s, slot, 2 * i, false);
+                            qk_chunk(d_s, slot + C::CHUNK, 2 * i + 1, false);
+                            progressed = true;
+                            if (++qstage > C::PAIRS) {
+                                umma_commit(bar(BR::SFULL + (kq & 1)));
+                                if (qc.last()) {
+                                    umma_commit(bar(BR::QEMPTY));
+                                    ++seg_q;
+                                }
+                                qc.advance(tile_off);
+                                ++kq;
+                                qstage = 0;
+                            }
+                        }
                     }
                 }
                 if (progressed) {
