@@ -165,6 +165,33 @@ __device__ __forceinline__ float warp_colreduce16(const float (&v)[16], int lane
     return op2<IS_MAX>(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
 }
 
+// Same for 8 values per lane: lane l ends with column col8(l); lanes l..l+3 (l % 4 == 0) share it.
+__device__ __forceinline__ int col8(int lane) {
+    return (((lane >> 4) & 1) << 2) | (((lane >> 3) & 1) << 1) | ((lane >> 2) & 1);
+}
+template <bool IS_MAX>
+__device__ __forceinline__ float warp_colreduce8(const float (&v)[8], int lane) {
+    float a4[4], a2[2];
+    bool up = (lane & 16) != 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float send = up ? v[j] : v[j + 4];
+        float keep = up ? v[j + 4] : v[j];
+        a4[j] = op2<IS_MAX>(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+    }
+    up = (lane & 8) != 0;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        float send = up ? a4[j] : a4[j + 2];
+        float keep = up ? a4[j + 2] : a4[j];
+        a2[j] = op2<IS_MAX>(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+    }
+    up = (lane & 4) != 0;
+    float a1 = op2<IS_MAX>(up ? a2[1] : a2[0], __shfl_xor_sync(0xffffffffu, up ? a2[0] : a2[1], 4));
+    a1 = op2<IS_MAX>(a1, __shfl_xor_sync(0xffffffffu, a1, 2));
+    return op2<IS_MAX>(a1, __shfl_xor_sync(0xffffffffu, a1, 1));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x = lo (low 16 bits), .y = hi
     return *reinterpret_cast<uint32_t *>(&v);

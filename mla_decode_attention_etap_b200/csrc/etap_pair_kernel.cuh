@@ -22,8 +22,9 @@
 //     two 64-column chunks plus an 8 KB slot for the 32 rope columns; tail
 //     rows zeroed);
 //   * warp 1 lane 0: tcgen05.mma issuer, S^T of tile k+1 before O^T of tile k;
-//   * warps 2..5: one TMEM lane (= one KV row) per thread; the column softmax
-//     reduces ACROSS threads; P^T goes to shared memory as bf16 hi | lo.
+//   * warps 2..9: one TMEM lane (= one KV row) and half of the columns per
+//     thread; the column softmax reduces ACROSS threads; P^T goes to shared
+//     memory as bf16 hi | lo.
 //
 // Every wait is bounded; see etap_common.cuh.
 #pragma once
@@ -120,7 +121,7 @@ __device__ __forceinline__ uint32_t swz_off(uint32_t r, uint32_t j, uint32_t pit
 }
 
 template <class C>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     etap_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_kvr,
                      const __grid_constant__ DecodeParams p) {
@@ -160,10 +161,10 @@ __global__ void __launch_bounds__(192, 1)
         mbar_init(bar(BR::QEMPTY), 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(BR::SFULL + i), 1);
-            mbar_init(bar(BR::SEMPTY + i), 4);
+            mbar_init(bar(BR::SEMPTY + i), 8);
         }
         for (int i = 0; i < C::PB; ++i) {
-            mbar_init(bar(BR::PFULL + i), 4);
+            mbar_init(bar(BR::PFULL + i), 8);
             mbar_init(bar(BR::PEMPTY + i), 1);
         }
         mbar_init(bar(BR::TAIL), 1);
@@ -171,7 +172,7 @@ __global__ void __launch_bounds__(192, 1)
         mbar_init(bar(BR::RED), 4);
         mbar_init(bar(BR::REDL), 4);
         for (int i = 0; i < C::XS; ++i) mbar_init(bar(BR::XFULL + i), 1);
-        mbar_init(bar(BR::XFREE), 4);
+        mbar_init(bar(BR::XFREE), 8);
         wc->abort = 0;
         wc->limit_ns = p.wait_limit_ns;
         fence_barrier_init();
@@ -480,12 +481,15 @@ __global__ void __launch_bounds__(192, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax + epilogue (warps 2..5)
-        // The four warps synchronise through named barrier 1; a failed (timed
-        // out) wait only clears this thread's `ok`, and the next bar.red turns
-        // that into a uniform stop, so no thread is left waiting at a barrier.
-        constexpr uint32_t SMX = 1, NSM = 128;
+        // ------------------------------------------------------------ softmax + epilogue (warps 2..9)
+        // Two warps per TMEM lane quadrant: the thread owning KV row `row` handles 8 of every 16
+        // columns (`half` picks which).  The eight warps synchronise through named barrier 1; a
+        // failed (timed out) wait only clears this thread's `ok`, and the next bar.red turns that
+        // into a uniform stop, so no thread is left waiting at a barrier.
+        constexpr uint32_t SMX = 1, NSM = 256;
+        constexpr int NH = NG / 2;  // columns of the group this thread handles
         const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int row = quad * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         float *red = reinterpret_cast<float *>(smem + C::OFF_RED);    // [2][4][16]
@@ -495,6 +499,8 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t xfree_remote = map_to_rank(bar(BR::XFREE), peer);
         const int k_total = (int)(fe - fb);
         bool ok = true, stop = false;
+        // Exchange slots hold 128 rows x 16 fp32; this thread's 8 values are 16-byte chunks 2*half, 2*half+1.
+        auto x_off = [&](int j) -> uint32_t { return swz_off(row, 2 * half + j, 64, 3); };
         // CH > 1: whole-tile exchange, one tile ahead.  Our partial S^T of tile kk goes to the
         // peer's slots 0..CH-1 once the peer has combined tile kk-1 (XFREE).
         auto send_tile = [&](int kk) {
@@ -503,14 +509,14 @@ __global__ void __launch_bounds__(192, 1)
             ok = ok && spin_phase<true>(bar(BR::XFREE), (kk & 1) ^ 1, wc, status);
 #pragma unroll
             for (int ch = 0; ch < C::CH; ++ch) {
-                float xs16[16];
-                tmem_ld16(tmem + lane_addr + C::S_COL + (kk & 1) * NG + 16 * ch, xs16);
+                float xs8[8];
+                tmem_ld8(tmem + lane_addr + C::S_COL + (kk & 1) * NG + 16 * ch + 8 * half, xs8);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 4 && ok; ++j)
-                    st_async_v4(x_remote + ch * C::X_SLOT + swz_off(row, j, 64, 3), __float_as_uint(xs16[4 * j]),
-                                __float_as_uint(xs16[4 * j + 1]), __float_as_uint(xs16[4 * j + 2]),
-                                __float_as_uint(xs16[4 * j + 3]), xfull_remote);
+                for (int j = 0; j < 2 && ok; ++j)
+                    st_async_v4(x_remote + ch * C::X_SLOT + x_off(j), __float_as_uint(xs8[4 * j]),
+                                __float_as_uint(xs8[4 * j + 1]), __float_as_uint(xs8[4 * j + 2]),
+                                __float_as_uint(xs8[4 * j + 3]), xfull_remote);
             }
         };
         if (fb < fe) {
@@ -521,9 +527,9 @@ __global__ void __launch_bounds__(192, 1)
                 int L = p.seqlens[b];
                 if ((int64_t)L > l_cap) L = (int)l_cap;
                 if (L < 0) L = 0;
-                float m[NG], lpart[NG];
+                float m[NH], lpart[NH];  // index 8*ch + n  <->  column 16*ch + 8*half + n
 #pragma unroll
-                for (int n = 0; n < NG; ++n) {
+                for (int n = 0; n < NH; ++n) {
                     m[n] = -INFINITY;
                     lpart[n] = 0.f;
                 }
@@ -540,24 +546,24 @@ __global__ void __launch_bounds__(192, 1)
                         // (a) add the peer's partial S^T of tile k into ours, in TMEM, and free its slots;
                         // (b) send our partial of tile k+1 so it travels while tile k's softmax runs.
                         if (k == 0) send_tile(0);
-                        if (row == 0) mbar_arrive_expect_tx(bar(BR::XFULL), C::CH * C::X_SLOT);
+                        if (row == 0 && half == 0) mbar_arrive_expect_tx(bar(BR::XFULL), C::CH * C::X_SLOT);
                         ok = ok && spin_phase<true>(bar(BR::XFULL), k & 1, wc, status);
 #pragma unroll
                         for (int ch = 0; ch < C::CH; ++ch) {
-                            float xo[16];
-                            const uint32_t taddr = tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch;
-                            tmem_ld16(taddr, xo);
+                            float xo[8];
+                            const uint32_t taddr = tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch + 8 * half;
+                            tmem_ld8(taddr, xo);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const float4 v = *reinterpret_cast<const float4 *>(smem + C::OFF_X + ch * C::X_SLOT +
-                                                                                   swz_off(row, j, 64, 3));
+                            for (int j = 0; j < 2; ++j) {
+                                const float4 v =
+                                    *reinterpret_cast<const float4 *>(smem + C::OFF_X + ch * C::X_SLOT + x_off(j));
                                 xo[4 * j] += v.x;
                                 xo[4 * j + 1] += v.y;
                                 xo[4 * j + 2] += v.z;
                                 xo[4 * j + 3] += v.w;
                             }
-                            tmem_st16(taddr, xo);
+                            tmem_st8(taddr, xo);
                         }
                         tmem_wait_st();
                         __syncwarp();
@@ -571,8 +577,8 @@ __global__ void __launch_bounds__(192, 1)
                     }
 #pragma unroll
                     for (int ch = 0; ch < C::CH; ++ch) {
-                        float x[16];
-                        tmem_ld16(tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch, x);
+                        float x[8];
+                        tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch + 8 * half, x);
                         tmem_wait_ld();
                         if (ch == C::CH - 1) {
                             tc_fence_before();
@@ -580,37 +586,37 @@ __global__ void __launch_bounds__(192, 1)
                             if (lane == 0) mbar_arrive(bar(BR::SEMPTY + (k & 1)));
                         }
                         if constexpr (C::CH == 1) {
-                        // ---- exchange of the partial scores with the peer CTA.  Slot xs is free for
-                        // exchange e without a handshake: the peer overwrites it (exchange e + XS) only
-                        // after receiving our exchange e + XS - 1, which we send after consuming e.
-                        static_assert(C::XS >= 2, "slot reuse relies on at least two exchange slots");
-                        const int xs = e % C::XS, xu = e / C::XS;
-                        ++e;
+                            // ---- exchange of the partial scores with the peer CTA.  Slot xs is free for
+                            // exchange e without a handshake: the peer overwrites it (exchange e + XS) only
+                            // after receiving our exchange e + XS - 1, which we send after consuming e.
+                            static_assert(C::XS >= 2, "slot reuse relies on at least two exchange slots");
+                            const int xs = e % C::XS, xu = e / C::XS;
+                            ++e;
 #pragma unroll
-                        for (int j = 0; j < 4 && ok; ++j)
-                            st_async_v4(x_remote + xs * C::X_SLOT + swz_off(row, j, 64, 3), __float_as_uint(x[4 * j]),
-                                        __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
-                                        __float_as_uint(x[4 * j + 3]), xfull_remote + 8u * xs);
-                        if (row == 0) mbar_arrive_expect_tx(bar(BR::XFULL + xs), C::X_SLOT);
-                        ok = ok && spin_phase<true>(bar(BR::XFULL + xs), xu & 1, wc, status);
+                            for (int j = 0; j < 2 && ok; ++j)
+                                st_async_v4(x_remote + xs * C::X_SLOT + x_off(j), __float_as_uint(x[4 * j]),
+                                            __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
+                                            __float_as_uint(x[4 * j + 3]), xfull_remote + 8u * xs);
+                            if (row == 0 && half == 0) mbar_arrive_expect_tx(bar(BR::XFULL + xs), C::X_SLOT);
+                            ok = ok && spin_phase<true>(bar(BR::XFULL + xs), xu & 1, wc, status);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float4 v = *reinterpret_cast<const float4 *>(smem + C::OFF_X + xs * C::X_SLOT +
-                                                                               swz_off(row, j, 64, 3));
-                            x[4 * j] += v.x;
-                            x[4 * j + 1] += v.y;
-                            x[4 * j + 2] += v.z;
-                            x[4 * j + 3] += v.w;
+                            for (int j = 0; j < 2; ++j) {
+                                const float4 v =
+                                    *reinterpret_cast<const float4 *>(smem + C::OFF_X + xs * C::X_SLOT + x_off(j));
+                                x[4 * j] += v.x;
+                                x[4 * j + 1] += v.y;
+                                x[4 * j + 2] += v.z;
+                                x[4 * j + 3] += v.w;
+                            }
                         }
-                        }  // CH == 1 exchange
                         // ---- scale + mask
                         if (full_tile) {
 #pragma unroll
-                            for (int n = 0; n < 16; ++n) x[n] *= p.scale_log2;
+                            for (int n = 0; n < 8; ++n) x[n] *= p.scale_log2;
                         } else {
 #pragma unroll
-                            for (int n = 0; n < 16; ++n) {
-                                const int ng = grp * NG + 16 * ch + n;
+                            for (int n = 0; n < 8; ++n) {
+                                const int ng = grp * NG + 16 * ch + 8 * half + n;
                                 int vis = 0;
                                 if (ng < p.ncols) {
                                     vis = p.causal ? (L - p.q_len + ng / p.num_heads + 1) : L;
@@ -622,60 +628,61 @@ __global__ void __launch_bounds__(192, 1)
                         // ---- running maximum: kept unless some row of the tile exceeds it by > 2^8
                         bool need = first || !ok;
 #pragma unroll
-                        for (int n = 0; n < 16; ++n) need = need || (x[n] > m[16 * ch + n] + kRescaleThreshold);
-                        float alpha[16];
+                        for (int n = 0; n < 8; ++n) need = need || (x[n] > m[8 * ch + n] + kRescaleThreshold);
+                        float alpha[8];
 #pragma unroll
-                        for (int n = 0; n < 16; ++n) alpha[n] = 1.f;
+                        for (int n = 0; n < 8; ++n) alpha[n] = 1.f;
                         bool rescale = false;
                         if (named_bar_or(SMX, NSM, need)) {
                             if (!named_bar_and(SMX, NSM, ok)) {
                                 stop = true;
                                 break;
                             }
-                            // column maximum of the tile: across lanes, then across the 4 warps
-                            const float wmax = warp_colreduce16<true>(x, lane);
+                            // column maximum of the tile: across lanes, then across the 4 quadrants
+                            const float wmax = warp_colreduce8<true>(x, lane);
                             float *rb = red + (red_uses & 1) * 64;
                             ++red_uses;
-                            if ((lane & 1) == 0) rb[quad * 16 + col16(lane)] = wmax;
+                            if ((lane & 3) == 0) rb[quad * 16 + 8 * half + col8(lane)] = wmax;
                             named_bar_sync(SMX, NSM);
 #pragma unroll
-                            for (int n4 = 0; n4 < 16; n4 += 4) {
-                                const float4 a = *reinterpret_cast<const float4 *>(rb + 0 * 16 + n4);
-                                const float4 bq = *reinterpret_cast<const float4 *>(rb + 1 * 16 + n4);
-                                const float4 c = *reinterpret_cast<const float4 *>(rb + 2 * 16 + n4);
-                                const float4 d = *reinterpret_cast<const float4 *>(rb + 3 * 16 + n4);
+                            for (int n4 = 0; n4 < 8; n4 += 4) {
+                                const int c0 = 8 * half + n4;
+                                const float4 a = *reinterpret_cast<const float4 *>(rb + 0 * 16 + c0);
+                                const float4 bq = *reinterpret_cast<const float4 *>(rb + 1 * 16 + c0);
+                                const float4 c = *reinterpret_cast<const float4 *>(rb + 2 * 16 + c0);
+                                const float4 d = *reinterpret_cast<const float4 *>(rb + 3 * 16 + c0);
                                 const float mt4[4] = {fmaxf(fmaxf(a.x, bq.x), fmaxf(c.x, d.x)),
                                                       fmaxf(fmaxf(a.y, bq.y), fmaxf(c.y, d.y)),
                                                       fmaxf(fmaxf(a.z, bq.z), fmaxf(c.z, d.z)),
                                                       fmaxf(fmaxf(a.w, bq.w), fmaxf(c.w, d.w))};
 #pragma unroll
                                 for (int u = 0; u < 4; ++u) {
-                                    const int n = n4 + u, cn = 16 * ch + n;
+                                    const int n = n4 + u, li = 8 * ch + n;
                                     if (first) {
-                                        m[cn] = mt4[u];
-                                    } else if (mt4[u] > m[cn] + kRescaleThreshold) {
-                                        alpha[n] = fast_exp2(m[cn] - mt4[u]);
-                                        m[cn] = mt4[u];
+                                        m[li] = mt4[u];
+                                    } else if (mt4[u] > m[li] + kRescaleThreshold) {
+                                        alpha[n] = fast_exp2(m[li] - mt4[u]);
+                                        m[li] = mt4[u];
                                         rescale = true;
                                     }
                                 }
                             }
                         }
-                        float pv[16];
+                        float pv[8];
 #pragma unroll
-                        for (int n = 0; n < 16; ++n) {
-                            const int cn = 16 * ch + n;
-                            const float mu = (m[cn] == -INFINITY) ? 0.f : m[cn];
+                        for (int n = 0; n < 8; ++n) {
+                            const int li = 8 * ch + n;
+                            const float mu = (m[li] == -INFINITY) ? 0.f : m[li];
                             pv[n] = fast_exp2(x[n] - mu);
-                            lpart[cn] = lpart[cn] * alpha[n] + pv[n];
+                            lpart[li] = lpart[li] * alpha[n] + pv[n];
                         }
-                        // ---- P^T row chunk -> shared memory: bf16 hi into columns [16ch, 16ch+16), lo into NG + that
+                        // ---- P^T row chunk -> shared memory: bf16 hi into column 16ch+8half.., lo into NG + that
                         if (ch == 0)
                             ok = ok && spin_phase<false>(bar(BR::PEMPTY + pb), ((k / C::PB) & 1) ^ 1, wc, status);
                         {
-                            uint32_t hi[8], lo[8];
+                            uint32_t hi[4], lo[4];
 #pragma unroll
-                            for (int n = 0; n < 16; n += 2) {
+                            for (int n = 0; n < 8; n += 2) {
                                 const __nv_bfloat16 h0 = __float2bfloat16_rn(pv[n]);
                                 const __nv_bfloat16 h1 = __float2bfloat16_rn(pv[n + 1]);
                                 hi[n / 2] =
@@ -684,17 +691,14 @@ __global__ void __launch_bounds__(192, 1)
                             }
                             uint8_t *pbuf = smem + C::OFF_P + pb * C::P_BUF;
 #pragma unroll
-                            for (int half = 0; half < 2; ++half) {
-                                const uint32_t *w = half == 0 ? hi : lo;
-                                const int col0 = half * NG + 16 * ch;  // first P^T column of these 16
+                            for (int hl = 0; hl < 2; ++hl) {
+                                const uint32_t *w = hl == 0 ? hi : lo;
+                                const int col0 = hl * NG + 16 * ch + 8 * half;  // first P^T column of these 8
                                 const int atom = col0 / C::AW;
                                 const int j0 = (col0 % C::AW) / 8;  // 16-byte chunk within the atom row
-#pragma unroll
-                                for (int jj = 0; jj < 2; ++jj) {
-                                    uint4 *dst = reinterpret_cast<uint4 *>(
-                                        pbuf + atom * C::P_ATOM + swz_off(row, j0 + jj, C::P_PITCH, C::P_SWZ_MASK));
-                                    *dst = make_uint4(w[4 * jj], w[4 * jj + 1], w[4 * jj + 2], w[4 * jj + 3]);
-                                }
+                                *reinterpret_cast<uint4 *>(pbuf + atom * C::P_ATOM +
+                                                           swz_off(row, j0, C::P_PITCH, C::P_SWZ_MASK)) =
+                                    make_uint4(w[0], w[1], w[2], w[3]);
                             }
                         }
                         if (rescale) {
@@ -702,7 +706,7 @@ __global__ void __launch_bounds__(192, 1)
                             if (!waited_prev) {
                                 const int kp = k - 1;
                                 ok = ok && spin_phase<false>(bar(BR::PEMPTY + (kp % C::PB)), (kp / C::PB) & 1, wc,
-                                                      status);
+                                                             status);
                                 tc_fence_after();
                                 waited_prev = true;
                             }
@@ -710,14 +714,15 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                             for (int i = 0; i < C::PAIRS; ++i) {
 #pragma unroll
-                                for (int half = 0; half < 2; ++half) {
-                                    float v[16];
-                                    const uint32_t addr = tmem + lane_addr + C::O_COL + i * C::NP + half * NG + 16 * ch;
-                                    tmem_ld16(addr, v);
+                                for (int hl = 0; hl < 2; ++hl) {
+                                    float v[8];
+                                    const uint32_t addr =
+                                        tmem + lane_addr + C::O_COL + i * C::NP + hl * NG + 16 * ch + 8 * half;
+                                    tmem_ld8(addr, v);
                                     tmem_wait_ld();
 #pragma unroll
-                                    for (int n = 0; n < 16; ++n) v[n] *= alpha[n];
-                                    tmem_st16(addr, v);
+                                    for (int n = 0; n < 8; ++n) v[n] *= alpha[n];
+                                    tmem_st8(addr, v);
                                 }
                             }
                         }
@@ -739,11 +744,11 @@ __global__ void __launch_bounds__(192, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int ch = 0; ch < C::CH; ++ch) {
-                    float v16[16];
+                    float v8[8];
 #pragma unroll
-                    for (int n = 0; n < 16; ++n) v16[n] = lpart[16 * ch + n];
-                    const float wsum = warp_colreduce16<false>(v16, lane);
-                    if ((lane & 1) == 0) redl[quad * NG + 16 * ch + col16(lane)] = wsum;
+                    for (int n = 0; n < 8; ++n) v8[n] = lpart[8 * ch + n];
+                    const float wsum = warp_colreduce8<false>(v8, lane);
+                    if ((lane & 3) == 0) redl[quad * NG + 16 * ch + 8 * half + col8(lane)] = wsum;
                 }
                 if (!named_bar_and(SMX, NSM, ok)) {  // also orders the redl writes before the reads
                     stop = true;
@@ -753,25 +758,25 @@ __global__ void __launch_bounds__(192, 1)
                 const int slot = seq_info[4 * b + 3] + (unit - seq_info[4 * b + 1]);
 #pragma unroll
                 for (int ch = 0; ch < C::CH; ++ch) {
-                    float inv_l[16], lse_n[16];
+                    float inv_l[8], lse_n[8];
 #pragma unroll
-                    for (int n = 0; n < 16; ++n) {
-                        const int cn = 16 * ch + n;
+                    for (int n = 0; n < 8; ++n) {
+                        const int cn = 16 * ch + 8 * half + n, li = 8 * ch + n;
                         const float l = redl[cn] + redl[NG + cn] + redl[2 * NG + cn] + redl[3 * NG + cn];
-                        const bool empty = !(l > 0.f) || m[cn] == -INFINITY;
+                        const bool empty = !(l > 0.f) || m[li] == -INFINITY;
                         inv_l[n] = empty ? 0.f : 1.f / l;
-                        lse_n[n] = empty ? -INFINITY : (m[cn] + __log2f(l)) * 0.69314718055994531f;
+                        lse_n[n] = empty ? -INFINITY : (m[li] + __log2f(l)) * 0.69314718055994531f;
                     }
 #pragma unroll
                     for (int i = 0; i < C::PAIRS; ++i) {
-                        float hi[16], lo[16];
-                        tmem_ld16(tmem + lane_addr + C::O_COL + i * C::NP + 16 * ch, hi);
-                        tmem_ld16(tmem + lane_addr + C::O_COL + i * C::NP + NG + 16 * ch, lo);
+                        float hi[8], lo[8];
+                        tmem_ld8(tmem + lane_addr + C::O_COL + i * C::NP + 16 * ch + 8 * half, hi);
+                        tmem_ld8(tmem + lane_addr + C::O_COL + i * C::NP + NG + 16 * ch + 8 * half, lo);
                         tmem_wait_ld();
                         const int d = 256 * (int)rank + 128 * i + row;
 #pragma unroll
-                        for (int n = 0; n < 16; ++n) {
-                            const int ng = grp * NG + 16 * ch + n;
+                        for (int n = 0; n < 8; ++n) {
+                            const int ng = grp * NG + 16 * ch + 8 * half + n;
                             if (ng >= p.ncols) continue;
                             const float val = (hi[n] + lo[n]) * inv_l[n];
                             if (nsplit == 1)
@@ -780,11 +785,11 @@ __global__ void __launch_bounds__(192, 1)
                                 p.opart[((int64_t)slot * p.ncols + ng) * kDv + d] = val;
                         }
                     }
-                    if (rank == 0 && quad == 0 && lane < 16) {
-                        const int ng = grp * NG + 16 * ch + lane;
+                    if (rank == 0 && quad == 0 && lane < 8) {
+                        const int ng = grp * NG + 16 * ch + 8 * half + lane;
                         float my = lse_n[0];
 #pragma unroll
-                        for (int n = 1; n < 16; ++n)
+                        for (int n = 1; n < 8; ++n)
                             if (lane == n) my = lse_n[n];
                         if (ng < p.ncols) {
                             if (nsplit == 1) p.lse[(int64_t)b * p.ncols + ng] = my;

@@ -103,7 +103,7 @@ cudaError_t launch_pair(const CUtensorMap &tm_q, const CUtensorMap &tm_kv, const
                         const CUtensorMap &tm_kvr, const mla::DecodeParams &p, int clusters, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * clusters, 1, 1);
-    cfg.blockDim = dim3(192, 1, 1);
+    cfg.blockDim = dim3(320, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_ALLOC;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
