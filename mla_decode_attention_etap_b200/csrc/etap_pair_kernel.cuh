@@ -84,9 +84,11 @@ struct PairCfg {
 };
 
 using PairCfg16 = PairCfg<16, 5, 2, 2>;  // h*q_len <= 16
-using PairCfg64 = PairCfg<64, 3, 2, 1>;  // 16 < h*q_len, in groups of 64 columns
+using PairCfg32 = PairCfg<32, 5, 1, 1>;  // 16 < h*q_len, in groups of 32 columns
+using PairCfg64 = PairCfg<64, 3, 2, 1>;  // groups of 64 columns (3-slot ring: fewer groups, less overlap)
 
-static_assert(PairCfg16::SMEM_ALLOC <= 232448 && PairCfg64::SMEM_ALLOC <= 232448, "shared memory plan > 227 KB");
+static_assert(PairCfg16::SMEM_ALLOC <= 232448 && PairCfg32::SMEM_ALLOC <= 232448 && PairCfg64::SMEM_ALLOC <= 232448,
+              "shared memory plan > 227 KB");
 static_assert(PairCfg16::TMEM_COLS <= 512 && PairCfg64::TMEM_COLS <= 512, "TMEM plan");
 static_assert(PairCfg16::OFF_P % 1024 == 0 && PairCfg64::OFF_P % 1024 == 0, "alignment");
 static_assert(PairCfg16::OFF_QR % 512 == 0 && PairCfg64::OFF_QR % 512 == 0, "alignment");

@@ -89,8 +89,8 @@ int ensure_smem_attr() {
         e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)mla::PairCfg16::SMEM_ALLOC);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-        e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)mla::PairCfg64::SMEM_ALLOC);
+        e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)mla::PairCfg32::SMEM_ALLOC);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         done[dev] = true;
     }
@@ -281,7 +281,7 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = ng == 16 ? launch_pair<mla::PairCfg16>(tm_q, tm_kv, tm_qr, tm_kvr, p, lay.ctas * lay.groups, s)
-                             : launch_pair<mla::PairCfg64>(tm_q, tm_kv, tm_qr, tm_kvr, p, lay.ctas * lay.groups, s);
+                             : launch_pair<mla::PairCfg32>(tm_q, tm_kv, tm_qr, tm_kvr, p, lay.ctas * lay.groups, s);
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");

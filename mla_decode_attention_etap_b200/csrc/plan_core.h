@@ -39,8 +39,8 @@ enum : int {
 };
 
 // Query columns (heads x tokens) per cluster = UMMA N of S^T: one group of 16
-// when they fit, otherwise groups of 64.
-MLA_HD int group_cols(int ncols) { return ncols <= 16 ? 16 : 64; }
+// when they fit, otherwise groups of 32 (whose kernel keeps a 5-slot ring).
+MLA_HD int group_cols(int ncols) { return ncols <= 16 ? 16 : 32; }
 MLA_HD int num_groups(int ncols) { return (ncols + group_cols(ncols) - 1) / group_cols(ncols); }
 // Work units per column group: one per pair of SMs (a 2-CTA cluster).
 MLA_HD int num_ctas(int num_sms, int groups) {

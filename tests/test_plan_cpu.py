@@ -22,7 +22,7 @@ def test_schedule_invariants(seed, n_sms, h, q):
     lens[rng.random(B) < 0.2] = 0
     ranges, info, ctas, groups = m.mla_decode_plan_host(lens, q, h, n_sms)
     ncols = q * h
-    assert groups == (1 if ncols <= 16 else (ncols + 63) // 64)
+    assert groups == (1 if ncols <= 16 else (ncols + 31) // 32)
     assert ctas == max(1, n_sms // 2 // groups)  # one work unit per SM pair
     T = sum(tiles(int(L)) for L in lens)
     # the CTA ranges tile [0, T) in order; the working CTAs come first, each with
