@@ -219,7 +219,7 @@ __device__ __forceinline__ bool spin_phase(uint32_t bar, uint32_t parity, volati
     }
 }
 
-// Bounded wait on a phase completed by the peer CTA of the cluster (acquire at cluster scope).
+// Bounded wait on a phase completed by the peer CTA of the cluster.
 __device__ __forceinline__ bool wait_phase_cluster(uint32_t bar, uint32_t parity, volatile WaitCtl *wc,
                                                    int32_t *status) {
     if (mbar_try_wait_cluster(bar, parity)) return true;

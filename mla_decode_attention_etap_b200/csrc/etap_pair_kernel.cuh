@@ -544,30 +544,33 @@ __global__ void __launch_bounds__(320, 1)
                     // every row of the tile visible to every column: no per-column mask needed
                     const bool full_tile = (t + 1) * kTileRows <= (p.causal ? L - p.q_len + 1 : L);
                     bool waited_prev = false, rescale_any = false, sent_next = false;
+                    float xc[C::CH][8];  // CH > 1: full scores of this thread's columns, in registers
                     if constexpr (C::CH > 1) {
-                        // (a) add the peer's partial S^T of tile k into ours, in TMEM, and free its slots;
-                        // (b) send our partial of tile k+1 so it travels while tile k's softmax runs.
+                        // (a) add the peer's partial S^T of tile k to ours in registers; free the TMEM
+                        //     buffer and the peer's slots; (b) send our partial of tile k+1 so it travels
+                        //     while tile k's softmax runs.
                         if (k == 0) send_tile(0);
+#pragma unroll
+                        for (int ch = 0; ch < C::CH; ++ch)
+                            tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch + 8 * half, xc[ch]);
+                        tmem_wait_ld();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(BR::SEMPTY + (k & 1)));
                         if (row == 0 && half == 0) mbar_arrive_expect_tx(bar(BR::XFULL), C::CH * C::X_SLOT);
                         ok = ok && spin_phase<true>(bar(BR::XFULL), k & 1, wc, status);
 #pragma unroll
                         for (int ch = 0; ch < C::CH; ++ch) {
-                            float xo[8];
-                            const uint32_t taddr = tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch + 8 * half;
-                            tmem_ld8(taddr, xo);
-                            tmem_wait_ld();
 #pragma unroll
                             for (int j = 0; j < 2; ++j) {
                                 const float4 v =
                                     *reinterpret_cast<const float4 *>(smem + C::OFF_X + ch * C::X_SLOT + x_off(j));
-                                xo[4 * j] += v.x;
-                                xo[4 * j + 1] += v.y;
-                                xo[4 * j + 2] += v.z;
-                                xo[4 * j + 3] += v.w;
+                                xc[ch][4 * j] += v.x;
+                                xc[ch][4 * j + 1] += v.y;
+                                xc[ch][4 * j + 2] += v.z;
+                                xc[ch][4 * j + 3] += v.w;
                             }
-                            tmem_st8(taddr, xo);
                         }
-                        tmem_wait_st();
                         __syncwarp();
                         if (lane == 0) mbar_arrive_remote(xfree_remote);
                         // Send now only if S^T of tile k+1 is already there: with few V slots its
@@ -580,9 +583,12 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                     for (int ch = 0; ch < C::CH; ++ch) {
                         float x[8];
-                        tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch + 8 * half, x);
-                        tmem_wait_ld();
-                        if (ch == C::CH - 1) {
+                        if constexpr (C::CH > 1) {
+#pragma unroll
+                            for (int n = 0; n < 8; ++n) x[n] = xc[ch][n];
+                        } else {
+                            tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch + 8 * half, x);
+                            tmem_wait_ld();
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(bar(BR::SEMPTY + (k & 1)));
