@@ -71,8 +71,8 @@ struct PairCfg {
     static constexpr uint32_t OFF_P = align1024(OFF_QR + Q_ROPE);
     static constexpr uint32_t OFF_X = OFF_P + PB * P_BUF;
     static constexpr uint32_t OFF_BAR = OFF_X + XS * X_SLOT;
-    static constexpr uint32_t OFF_RED = OFF_BAR + 512;                 // float [2][4][16] column max exchange
-    static constexpr uint32_t OFF_REDL = OFF_RED + 512;                // float [4][NG] column sum exchange
+    static constexpr uint32_t OFF_RED = OFF_BAR + 512;                 // float [2][4][NG] column max exchange
+    static constexpr uint32_t OFF_REDL = OFF_RED + 32 * NG;               // float [4][NG] column sum exchange
     static constexpr uint32_t OFF_MISC = OFF_REDL + 16 * NG;
     static constexpr uint32_t BYTES = OFF_MISC + 64;
     static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;               // slack for 1024-byte alignment
@@ -85,13 +85,11 @@ struct PairCfg {
 
 using PairCfg16 = PairCfg<16, 5, 2, 2>;  // h*q_len <= 16
 using PairCfg32 = PairCfg<32, 5, 1, 1>;  // 16 < h*q_len, in groups of 32 columns
-using PairCfg64 = PairCfg<64, 3, 2, 1>;  // groups of 64 columns (3-slot ring: fewer groups, less overlap)
 
-static_assert(PairCfg16::SMEM_ALLOC <= 232448 && PairCfg32::SMEM_ALLOC <= 232448 && PairCfg64::SMEM_ALLOC <= 232448,
-              "shared memory plan > 227 KB");
-static_assert(PairCfg16::TMEM_COLS <= 512 && PairCfg64::TMEM_COLS <= 512, "TMEM plan");
-static_assert(PairCfg16::OFF_P % 1024 == 0 && PairCfg64::OFF_P % 1024 == 0, "alignment");
-static_assert(PairCfg16::OFF_QR % 512 == 0 && PairCfg64::OFF_QR % 512 == 0, "alignment");
+static_assert(PairCfg16::SMEM_ALLOC <= 232448 && PairCfg32::SMEM_ALLOC <= 232448, "shared memory plan > 227 KB");
+static_assert(PairCfg16::TMEM_COLS <= 512 && PairCfg32::TMEM_COLS <= 512, "TMEM plan");
+static_assert(PairCfg16::OFF_P % 1024 == 0 && PairCfg32::OFF_P % 1024 == 0, "alignment");
+static_assert(PairCfg16::OFF_QR % 512 == 0 && PairCfg32::OFF_QR % 512 == 0, "alignment");
 
 template <class C>
 struct PairBars {
@@ -109,11 +107,14 @@ struct PairBars {
     static constexpr int FINAL = TAIL + 1;
     static constexpr int RED = FINAL + 1;
     static constexpr int REDL = RED + 1;
-    static constexpr int XFULL = REDL + 1;
-    static constexpr int XFREE = XFULL + C::XS;  // used when CH > 1: the peer consumed our last tile
-    static constexpr int COUNT = XFREE + 1;
+    // Exchange barriers are per softmax warp: warp w only needs (and only frees) the partial
+    // scores of the peer's warp w (same rows, same columns), and one barrier per warp keeps the
+    // transaction counts of the 16-byte remote stores off a single shared barrier.
+    static constexpr int XFULL = REDL + 1;       // [XS][8]
+    static constexpr int XFREE = XFULL + 8 * C::XS;  // [8], used when CH > 1: the peer consumed our last tile
+    static constexpr int COUNT = XFREE + 8;
 };
-static_assert(PairBars<PairCfg16>::COUNT * 8 <= 512 && PairBars<PairCfg64>::COUNT * 8 <= 512, "barrier area");
+static_assert(PairBars<PairCfg16>::COUNT * 8 <= 512 && PairBars<PairCfg32>::COUNT * 8 <= 512, "barrier area");
 
 // Byte offset of 16-byte chunk j of row r in a row-major buffer of `pitch`-byte
 // rows swizzled like the MMA operand (chunk index XOR address bits 7+).
@@ -173,8 +174,8 @@ __global__ void __launch_bounds__(320, 1)
         mbar_init(bar(BR::FINAL), 1);
         mbar_init(bar(BR::RED), 4);
         mbar_init(bar(BR::REDL), 4);
-        for (int i = 0; i < C::XS; ++i) mbar_init(bar(BR::XFULL + i), 1);
-        mbar_init(bar(BR::XFREE), 8);
+        for (int i = 0; i < 8 * C::XS; ++i) mbar_init(bar(BR::XFULL + i), 1);
+        for (int i = 0; i < 8; ++i) mbar_init(bar(BR::XFREE + i), 1);
         wc->abort = 0;
         wc->limit_ns = p.wait_limit_ns;
         fence_barrier_init();
@@ -494,11 +495,12 @@ __global__ void __launch_bounds__(320, 1)
         const int half = (warp - 2) >> 2;
         const int row = quad * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        float *red = reinterpret_cast<float *>(smem + C::OFF_RED);    // [2][4][16]
+        float *red = reinterpret_cast<float *>(smem + C::OFF_RED);    // [2][4][NG]
         float *redl = reinterpret_cast<float *>(smem + C::OFF_REDL);  // [4][NG]
         const uint32_t x_remote = map_to_rank(sbase + C::OFF_X, peer);
-        const uint32_t xfull_remote = map_to_rank(bar(BR::XFULL), peer);
-        const uint32_t xfree_remote = map_to_rank(bar(BR::XFREE), peer);
+        const int sw = warp - 2;  // softmax warp index: its exchange barriers
+        const uint32_t xfull_remote = map_to_rank(bar(BR::XFULL + sw), peer);
+        const uint32_t xfree_remote = map_to_rank(bar(BR::XFREE + sw), peer);
         const int k_total = (int)(fe - fb);
         bool ok = true, stop = false;
         // Exchange slots hold 128 rows x 16 fp32; this thread's 8 values are 16-byte chunks 2*half, 2*half+1.
@@ -508,7 +510,7 @@ __global__ void __launch_bounds__(320, 1)
         auto send_tile = [&](int kk) {
             ok = ok && spin_phase<false>(bar(BR::SFULL + (kk & 1)), (kk >> 1) & 1, wc, status);
             tc_fence_after();
-            ok = ok && spin_phase<true>(bar(BR::XFREE), (kk & 1) ^ 1, wc, status);
+            ok = ok && spin_phase<true>(bar(BR::XFREE + sw), (kk & 1) ^ 1, wc, status);
 #pragma unroll
             for (int ch = 0; ch < C::CH; ++ch) {
                 float xs8[8];
@@ -557,8 +559,8 @@ __global__ void __launch_bounds__(320, 1)
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(BR::SEMPTY + (k & 1)));
-                        if (row == 0 && half == 0) mbar_arrive_expect_tx(bar(BR::XFULL), C::CH * C::X_SLOT);
-                        ok = ok && spin_phase<true>(bar(BR::XFULL), k & 1, wc, status);
+                        if (lane == 0) mbar_arrive_expect_tx(bar(BR::XFULL + sw), C::CH * C::X_SLOT / 8);
+                        ok = ok && spin_phase<true>(bar(BR::XFULL + sw), k & 1, wc, status);
 #pragma unroll
                         for (int ch = 0; ch < C::CH; ++ch) {
 #pragma unroll
@@ -580,21 +582,18 @@ __global__ void __launch_bounds__(320, 1)
                             sent_next = true;
                         }
                     }
+                    // ---- pass 1: full scores of this thread's columns (exchange for CH == 1), scale + mask
+                    bool need = first || !ok;
 #pragma unroll
                     for (int ch = 0; ch < C::CH; ++ch) {
-                        float x[8];
-                        if constexpr (C::CH > 1) {
-#pragma unroll
-                            for (int n = 0; n < 8; ++n) x[n] = xc[ch][n];
-                        } else {
-                            tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * NG + 16 * ch + 8 * half, x);
+                        float(&x)[8] = xc[ch];
+                        if constexpr (C::CH == 1) {
+                            tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * NG + 8 * half, x);
                             tmem_wait_ld();
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(bar(BR::SEMPTY + (k & 1)));
-                        }
-                        if constexpr (C::CH == 1) {
-                            // ---- exchange of the partial scores with the peer CTA.  Slot xs is free for
+                            // Exchange of the partial scores with the peer CTA.  Slot xs is free for
                             // exchange e without a handshake: the peer overwrites it (exchange e + XS) only
                             // after receiving our exchange e + XS - 1, which we send after consuming e.
                             static_assert(C::XS >= 2, "slot reuse relies on at least two exchange slots");
@@ -604,9 +603,9 @@ __global__ void __launch_bounds__(320, 1)
                             for (int j = 0; j < 2 && ok; ++j)
                                 st_async_v4(x_remote + xs * C::X_SLOT + x_off(j), __float_as_uint(x[4 * j]),
                                             __float_as_uint(x[4 * j + 1]), __float_as_uint(x[4 * j + 2]),
-                                            __float_as_uint(x[4 * j + 3]), xfull_remote + 8u * xs);
-                            if (row == 0 && half == 0) mbar_arrive_expect_tx(bar(BR::XFULL + xs), C::X_SLOT);
-                            ok = ok && spin_phase<true>(bar(BR::XFULL + xs), xu & 1, wc, status);
+                                            __float_as_uint(x[4 * j + 3]), xfull_remote + 64u * xs);
+                            if (lane == 0) mbar_arrive_expect_tx(bar(BR::XFULL + 8 * xs + sw), C::X_SLOT / 8);
+                            ok = ok && spin_phase<true>(bar(BR::XFULL + 8 * xs + sw), xu & 1, wc, status);
 #pragma unroll
                             for (int j = 0; j < 2; ++j) {
                                 const float4 v =
@@ -617,7 +616,6 @@ __global__ void __launch_bounds__(320, 1)
                                 x[4 * j + 3] += v.w;
                             }
                         }
-                        // ---- scale + mask
                         if (full_tile) {
 #pragma unroll
                             for (int n = 0; n < 8; ++n) x[n] *= p.scale_log2;
@@ -633,32 +631,39 @@ __global__ void __launch_bounds__(320, 1)
                                 x[n] = (rg < vis) ? x[n] * p.scale_log2 : -INFINITY;
                             }
                         }
-                        // ---- running maximum: kept unless some row of the tile exceeds it by > 2^8
-                        bool need = first || !ok;
+                        // running maximum: kept unless some row of the tile exceeds it by > 2^8
 #pragma unroll
                         for (int n = 0; n < 8; ++n) need = need || (x[n] > m[8 * ch + n] + kRescaleThreshold);
-                        float alpha[8];
+                    }
+                    // ---- one vote per tile; the slow path takes the column maxima of all chunks
+                    float alpha[C::CH][8];
+                    bool rescale = false;
 #pragma unroll
-                        for (int n = 0; n < 8; ++n) alpha[n] = 1.f;
-                        bool rescale = false;
-                        if (named_bar_or(SMX, NSM, need)) {
-                            if (!named_bar_and(SMX, NSM, ok)) {
-                                stop = true;
-                                break;
-                            }
-                            // column maximum of the tile: across lanes, then across the 4 quadrants
-                            const float wmax = warp_colreduce8<true>(x, lane);
-                            float *rb = red + (red_uses & 1) * 64;
-                            ++red_uses;
-                            if ((lane & 3) == 0) rb[quad * 16 + 8 * half + col8(lane)] = wmax;
-                            named_bar_sync(SMX, NSM);
+                    for (int ch = 0; ch < C::CH; ++ch)
+#pragma unroll
+                        for (int n = 0; n < 8; ++n) alpha[ch][n] = 1.f;
+                    if (named_bar_or(SMX, NSM, need)) {
+                        if (!named_bar_and(SMX, NSM, ok)) {
+                            stop = true;
+                            break;
+                        }
+                        float *rb = red + (red_uses & 1) * (4 * NG);  // [4 quadrants][NG columns]
+                        ++red_uses;
+#pragma unroll
+                        for (int ch = 0; ch < C::CH; ++ch) {
+                            const float wmax = warp_colreduce8<true>(xc[ch], lane);
+                            if ((lane & 3) == 0) rb[quad * NG + 16 * ch + 8 * half + col8(lane)] = wmax;
+                        }
+                        named_bar_sync(SMX, NSM);
+#pragma unroll
+                        for (int ch = 0; ch < C::CH; ++ch) {
 #pragma unroll
                             for (int n4 = 0; n4 < 8; n4 += 4) {
-                                const int c0 = 8 * half + n4;
-                                const float4 a = *reinterpret_cast<const float4 *>(rb + 0 * 16 + c0);
-                                const float4 bq = *reinterpret_cast<const float4 *>(rb + 1 * 16 + c0);
-                                const float4 c = *reinterpret_cast<const float4 *>(rb + 2 * 16 + c0);
-                                const float4 d = *reinterpret_cast<const float4 *>(rb + 3 * 16 + c0);
+                                const int c0 = 16 * ch + 8 * half + n4;
+                                const float4 a = *reinterpret_cast<const float4 *>(rb + 0 * NG + c0);
+                                const float4 bq = *reinterpret_cast<const float4 *>(rb + 1 * NG + c0);
+                                const float4 c = *reinterpret_cast<const float4 *>(rb + 2 * NG + c0);
+                                const float4 d = *reinterpret_cast<const float4 *>(rb + 3 * NG + c0);
                                 const float mt4[4] = {fmaxf(fmaxf(a.x, bq.x), fmaxf(c.x, d.x)),
                                                       fmaxf(fmaxf(a.y, bq.y), fmaxf(c.y, d.y)),
                                                       fmaxf(fmaxf(a.z, bq.z), fmaxf(c.z, d.z)),
@@ -669,20 +674,24 @@ __global__ void __launch_bounds__(320, 1)
                                     if (first) {
                                         m[li] = mt4[u];
                                     } else if (mt4[u] > m[li] + kRescaleThreshold) {
-                                        alpha[n] = fast_exp2(m[li] - mt4[u]);
+                                        alpha[ch][n] = fast_exp2(m[li] - mt4[u]);
                                         m[li] = mt4[u];
                                         rescale = true;
                                     }
                                 }
                             }
                         }
+                    }
+                    // ---- pass 2: probabilities, P^T (hi + lo) into shared memory, O^T rescale
+#pragma unroll
+                    for (int ch = 0; ch < C::CH; ++ch) {
                         float pv[8];
 #pragma unroll
                         for (int n = 0; n < 8; ++n) {
                             const int li = 8 * ch + n;
                             const float mu = (m[li] == -INFINITY) ? 0.f : m[li];
-                            pv[n] = fast_exp2(x[n] - mu);
-                            lpart[li] = lpart[li] * alpha[n] + pv[n];
+                            pv[n] = fast_exp2(xc[ch][n] - mu);
+                            lpart[li] = lpart[li] * alpha[ch][n] + pv[n];
                         }
                         // ---- P^T row chunk -> shared memory: bf16 hi into column 16ch+8half.., lo into NG + that
                         if (ch == 0)
@@ -729,7 +738,7 @@ __global__ void __launch_bounds__(320, 1)
                                     tmem_ld8(addr, v);
                                     tmem_wait_ld();
 #pragma unroll
-                                    for (int n = 0; n < 8; ++n) v[n] *= alpha[n];
+                                    for (int n = 0; n < 8; ++n) v[n] *= alpha[ch][n];
                                     tmem_st8(addr, v);
                                 }
                             }
