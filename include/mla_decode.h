@@ -100,7 +100,12 @@ MLA_API int mla_decode_plan(const int32_t *seqlens, int batch, int q_len, int nu
 
 /*
  * The decode itself (ETAP steps 1-4 of the pages, plus the split-KV partial
- * outputs and, unless MLA_FLAG_SKIP_COMBINE is set, the combine).
+ * outputs and, unless MLA_FLAG_SKIP_COMBINE is set, their merge).  Without that
+ * flag the merge runs inside the decode kernel: the last CTA to finish a split
+ * of a sequence merges all of its splits (same arithmetic as mla_combine, so the
+ * results are bitwise equal), and sequences with L_b = 0 get O = 0, LSE = -inf.
+ * (When num_sms allows more splits per sequence than the kernel's merge buffer
+ * holds, fwd launches the combine kernel after the decode instead.)
  *   q            bf16 [batch, q_len, num_heads, 576], 16-byte aligned
  *   kv           contiguous: bf16 [batch, kv_rows, 576];
  *                paged (block_table != NULL): bf16 [kv_rows / 64, 64, 576], i.e. kv_rows = num_blocks*64

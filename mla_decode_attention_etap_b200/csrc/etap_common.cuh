@@ -41,6 +41,9 @@ struct DecodeParams {
     unsigned long long wait_limit_ns;
     int withhold_q;    // test hook: never load Q, so that the bounded waits expire
     int cta_ranges_off, tile_off_off, seq_info_off;  // int32 offsets into ws
+    int32_t *counters;  // [batch][groups][2]: split CTAs done per (sequence, column group, rank)
+    int slots;          // partial slots (stride between the two ranks' LSE partial arrays)
+    int fuse_merge;     // the last split CTA of a sequence merges the partials (no combine launch)
 };
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA abort

@@ -30,6 +30,7 @@
 #pragma once
 
 #include "etap_common.cuh"
+#include "merge.cuh"
 
 namespace mla {
 
@@ -81,6 +82,8 @@ struct PairCfg {
     static constexpr uint32_t TMEM_COLS = pow2_at_least(2 * NP + 2 * NG);
     static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, NG, 0, 0);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, NP, 1, 1);
+    // The in-kernel split merge stages (splits + 1) x NG floats in the idle P^T buffers.
+    static constexpr int MERGE_MAX_SPLITS = (int)(PB * P_BUF / 4) / NG - 1;
 };
 
 using PairCfg16 = PairCfg<16, 5, 2, 2>;  // h*q_len <= 16
@@ -802,20 +805,116 @@ __global__ void __launch_bounds__(320, 1)
                                 p.opart[((int64_t)slot * p.ncols + ng) * kDv + d] = val;
                         }
                     }
-                    if (rank == 0 && quad == 0 && lane < 8) {
+                    if (quad == 0 && lane < 8) {
                         const int ng = grp * NG + 16 * ch + 8 * half + lane;
                         float my = lse_n[0];
 #pragma unroll
                         for (int n = 1; n < 8; ++n)
                             if (lane == n) my = lse_n[n];
                         if (ng < p.ncols) {
-                            if (nsplit == 1) p.lse[(int64_t)b * p.ncols + ng] = my;
-                            else p.lsepart[(int64_t)slot * p.ncols + ng] = my;
+                            if (nsplit == 1) {
+                                if (rank == 0) p.lse[(int64_t)b * p.ncols + ng] = my;
+                            } else {
+                                p.lsepart[((int64_t)rank * p.slots + slot) * p.ncols + ng] = my;
+                            }
                         }
+                    }
+                }
+                if (nsplit >= 2 && p.fuse_merge) {
+                    // Split-KV merge in the kernel: the last CTA (of this rank) to finish a split of
+                    // sequence b merges all splits for its 256 latent rows and this column group.
+                    // Release the partials of all 256 threads (ordered before the fence by the
+                    // barrier), count this split, and acquire the others' if it was the last one.
+                    named_bar_sync(SMX, NSM);
+                    volatile int *merge_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 32);
+                    int32_t *cnt = p.counters + ((int64_t)b * p.groups + grp) * 2 + rank;
+                    if (row == 0 && half == 0) {
+                        __threadfence();
+                        const bool last = atomicAdd(cnt, 1) == nsplit - 1;
+                        if (last) __threadfence();
+                        *merge_flag = last;
+                    }
+                    named_bar_sync(SMX, NSM);
+                    if (*merge_flag) {
+                        // thread = 4 consecutive latent rows (one float4) x NG/4 columns.  The first
+                        // U splits' partial outputs are in flight while the LSE partials are staged in
+                        // the idle P^T buffers (the last step 3 has completed) and merged per column.
+                        constexpr int NQ = NG / 4, U = 16 / NQ;
+                        const int s0 = seq_info[4 * b + 3];
+                        const int tid = (warp - 2) * 32 + lane;
+                        const int d4 = 256 * (int)rank + 4 * (tid & 63), nq0 = (tid >> 6) * NQ;
+                        const int nn = p.ncols - grp * NG < NG ? p.ncols - grp * NG : NG;
+                        const float *op = p.opart + ((int64_t)s0 * p.ncols + grp * NG + nq0) * kDv + d4;
+                        float *ls = reinterpret_cast<float *>(smem + C::OFF_P);  // [nsplit][NG]
+                        float *lt = ls + nsplit * NG;                             // [NG]
+                        float4 v[U][NQ];
+                        auto load_batch = [&](int sp0) {
+#pragma unroll
+                            for (int u = 0; u < U; ++u)
+#pragma unroll
+                                for (int j = 0; j < NQ; ++j)
+                                    v[u][j] = (sp0 + u < nsplit && nq0 + j < nn)
+                                                  ? __ldcg(reinterpret_cast<const float4 *>(
+                                                        op + ((int64_t)(sp0 + u) * p.ncols + j) * kDv))
+                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                        };
+                        load_batch(0);
+                        const float *lsrc = p.lsepart + ((int64_t)rank * p.slots + s0) * p.ncols + grp * NG;
+                        for (int i = tid; i < nsplit * NG; i += NSM) {
+                            const int sp = i / NG, n = i - sp * NG;
+                            ls[i] = grp * NG + n < p.ncols ? __ldcg(lsrc + (int64_t)sp * p.ncols + n) : -INFINITY;
+                        }
+                        named_bar_sync(SMX, NSM);
+                        if (tid < NG) lt[tid] = merged_lse([&](int sp) { return ls[sp * NG + tid]; }, nsplit);
+                        named_bar_sync(SMX, NSM);
+                        float acc[NQ][4];
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+                        for (int sp0 = 0; sp0 < nsplit; sp0 += U) {
+                            if (sp0 > 0) load_batch(sp0);
+#pragma unroll
+                            for (int u = 0; u < U; ++u)
+#pragma unroll
+                                for (int j = 0; j < NQ; ++j) {
+                                    const float lv = lt[nq0 + j];
+                                    if (sp0 + u < nsplit && nq0 + j < nn && lv != -INFINITY) {
+                                        const float w = merge_weight(ls[(sp0 + u) * NG + nq0 + j], lv);
+                                        acc[j][0] = fmaf(w, v[u][j].x, acc[j][0]);
+                                        acc[j][1] = fmaf(w, v[u][j].y, acc[j][1]);
+                                        acc[j][2] = fmaf(w, v[u][j].z, acc[j][2]);
+                                        acc[j][3] = fmaf(w, v[u][j].w, acc[j][3]);
+                                    }
+                                }
+                        }
+#pragma unroll
+                        for (int j = 0; j < NQ; ++j) {
+                            if (nq0 + j >= nn) break;
+                            const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[j][0], acc[j][1]);
+                            const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[j][2], acc[j][3]);
+                            uint2 packed;
+                            packed.x = *reinterpret_cast<const uint32_t *>(&lo);
+                            packed.y = *reinterpret_cast<const uint32_t *>(&hi);
+                            *reinterpret_cast<uint2 *>(p.o + ((int64_t)b * p.ncols + grp * NG + nq0 + j) * kDv + d4) = packed;
+                            if (rank == 0 && (tid & 63) == 0) p.lse[(int64_t)b * p.ncols + grp * NG + nq0 + j] = lt[nq0 + j];
+                        }
+                        // ls/lt are next overwritten as P^T after the next tile's vote barrier
+                        if (row == 0 && half == 0) *cnt = 0;  // ready for the next call
                     }
                 }
                 tc_fence_before();
                 ++seg;
+            }
+        }
+        if (p.fuse_merge && !stop && ok) {
+            // Sequences without a single KV row get no split: O = 0 and LSE = -inf, written by
+            // cluster b mod (number of clusters), each CTA for its 256 latent rows.
+            const int ncl = (int)(gridDim.x >> 1);
+            const int d = 256 * (int)rank + (warp - 2) * 32 + lane;
+            for (int bb = (int)(blockIdx.x >> 1); bb < p.batch; bb += ncl) {
+                if (seq_info[4 * bb + 2] != 0) continue;
+                for (int n = 0; n < p.ncols; ++n) p.o[((int64_t)bb * p.ncols + n) * kDv + d] = __float2bfloat16_rn(0.f);
+                if (rank == 0 && warp == 2)
+                    for (int n = lane; n < p.ncols; n += 32) p.lse[(int64_t)bb * p.ncols + n] = -INFINITY;
             }
         }
         if (stop || !ok) wc->abort = 1;

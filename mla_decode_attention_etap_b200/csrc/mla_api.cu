@@ -278,6 +278,12 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
     p.cta_ranges_off = (int)(lay.cta_ranges / 4);
     p.tile_off_off = (int)(lay.tile_off / 4);
     p.seq_info_off = (int)(lay.seq_info / 4);
+    p.counters = reinterpret_cast<int32_t *>(ws + lay.counters);
+    p.slots = lay.slots;
+    // splits of a sequence are at most the work units (CTA pairs per column group)
+    const int max_splits = ng == 16 ? mla::PairCfg16::MERGE_MAX_SPLITS : mla::PairCfg32::MERGE_MAX_SPLITS;
+    const bool separate_combine = !(flags & MLA_FLAG_SKIP_COMBINE) && lay.ctas > max_splits;
+    p.fuse_merge = ((flags & MLA_FLAG_SKIP_COMBINE) || separate_combine) ? 0 : 1;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = ng == 16 ? launch_pair<mla::PairCfg16>(tm_q, tm_kv, tm_qr, tm_kvr, p, lay.ctas * lay.groups, s)
@@ -285,8 +291,7 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
-    if (!(flags & MLA_FLAG_SKIP_COMBINE))
-        return mla_combine(workspace, batch, q_len, num_heads, num_sms, o, lse, stream);
+    if (separate_combine) return mla_combine(workspace, batch, q_len, num_heads, num_sms, o, lse, stream);
     return MLA_OK;
 }
 

@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "merge.cuh"
 #include "plan_core.h"
 
 namespace mla {
@@ -31,6 +32,8 @@ __global__ void plan_kernel(const int32_t *__restrict__ seqlens, int batch, int 
         ranges[2 * c] = (int32_t)cta_begin(total, used, c);
         ranges[2 * c + 1] = (int32_t)cta_begin(total, used, c + 1);
     }
+    int32_t *counters = ws + lay.counters / 4;
+    for (int i = threadIdx.x; i < 2 * batch * groups; i += blockDim.x) counters[i] = 0;
     for (int b = threadIdx.x; b < batch; b += blockDim.x) {
         const int t0 = tile_off[b], t1 = tile_off[b + 1];
         int first = -1, nsplit = 0;
@@ -73,20 +76,17 @@ __global__ void __launch_bounds__(128) combine_kernel(const int32_t *__restrict_
     float lse_tot = -INFINITY;
     if (nsplit >= 2) {
         const int s0 = seq_info[4 * b + 3];
-        float mx = -INFINITY;
-        for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, lsepart[(int64_t)(s0 + s) * ncols + n]);
-        if (mx != -INFINITY) {
-            float sum = 0.f;
-            for (int s = 0; s < nsplit; ++s) sum += expf(lsepart[(int64_t)(s0 + s) * ncols + n] - mx);
-            lse_tot = mx + logf(sum);
+        const float *l = lsepart + (int64_t)s0 * ncols + n;
+        lse_tot = merged_lse([&](int s) { return __ldcg(l + (int64_t)s * ncols); }, nsplit);
+        if (lse_tot != -INFINITY) {
             for (int s = 0; s < nsplit; ++s) {
-                const float w = expf(lsepart[(int64_t)(s0 + s) * ncols + n] - lse_tot);
-                const float4 v = *reinterpret_cast<const float4 *>(opart + ((int64_t)(s0 + s) * ncols + n) * kDv +
-                                                                   4 * threadIdx.x);
-                acc[0] += w * v.x;
-                acc[1] += w * v.y;
-                acc[2] += w * v.z;
-                acc[3] += w * v.w;
+                const float w = merge_weight(__ldcg(l + (int64_t)s * ncols), lse_tot);
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(opart + ((int64_t)(s0 + s) * ncols + n) * kDv +
+                                                                          4 * threadIdx.x));
+                acc[0] = fmaf(w, v.x, acc[0]);
+                acc[1] = fmaf(w, v.y, acc[1]);
+                acc[2] = fmaf(w, v.z, acc[2]);
+                acc[3] = fmaf(w, v.w, acc[3]);
             }
         }
     }

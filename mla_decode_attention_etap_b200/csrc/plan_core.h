@@ -67,7 +67,8 @@ struct WsLayout {
     size_t tile_off;    // int32 [batch + 1]
     size_t seq_info;    // int32 [batch][4]: tiles, first CTA, splits, slot offset
     size_t opart;       // fp32  [slots][ncols][512]
-    size_t lsepart;     // fp32  [slots][ncols]
+    size_t lsepart;     // fp32  [2 ranks][slots][ncols] (the two CTAs of a pair compute equal values)
+    size_t counters;    // int32 [batch][groups][2 ranks]: split CTAs done, for the in-kernel merge
     size_t total;
     int ctas, groups, slots;
 };
@@ -88,7 +89,9 @@ MLA_HD WsLayout ws_layout(int batch, int q_len, int num_heads, int num_sms) {
     w.opart = off;
     off += align256(sizeof(float) * (size_t)w.slots * ncols * kDv);
     w.lsepart = off;
-    off += align256(sizeof(float) * (size_t)w.slots * ncols);
+    off += align256(sizeof(float) * 2 * (size_t)w.slots * ncols);
+    w.counters = off;
+    off += align256(sizeof(int32_t) * 2 * (size_t)batch * w.groups);
     w.total = off;
     return w;
 }

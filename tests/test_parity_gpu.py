@@ -68,7 +68,7 @@ def test_mixed_lengths_with_empty_sequence_and_nan_padding():
     assert_parity(o, lse, o_ref, lse_ref, what="mixed")
 
 
-@pytest.mark.parametrize("n_sms", [1, 3, 16, 148, 300])
+@pytest.mark.parametrize("n_sms", [1, 3, 16, 148, 300, 1024])
 def test_split_counts(n_sms):
     """From one CTA walking every sequence to many CTAs per sequence (split + combine)."""
     w = W.make_workload(3, 16, [3000, 257, 1536], seed=4)
@@ -206,3 +206,37 @@ def test_bounded_waits_report_timeout_and_context_survives():
     w2 = W.make_workload(1, 128, [500], seed=16)
     _, _, st3, _ = run_cuda(w2, flags=FLAG_TEST_EXPIRE_WAITS, poison=False)
     assert st3 == -6
+
+
+@pytest.mark.parametrize("heads", [16, 128])
+def test_in_kernel_merge_matches_combine_and_resets_counters(heads):
+    """The decode kernel merges split-KV partials itself (the last split CTA of a sequence does
+    it): bitwise equal to decode-with-partials + the separate combine kernel, including empty
+    sequences, and repeatable without a new plan (the merge counters reset themselves)."""
+    from mla_decode_attention_etap_b200 import FLAG_SKIP_COMBINE, mla_combine
+    lens = [0, 5000, 1, 2900, 0, 777]
+    w = W.make_workload(len(lens), heads, lens, seed=17, paged=heads == 128)
+    dev = torch.device("cuda")
+    q, kv, sl = w.q.to(dev), w.kv.to(dev), w.seqlens.to(dev)
+    bt = w.block_table.to(dev) if w.block_table is not None else None
+    from mla_decode_attention_etap_b200 import MlaDecoder
+    dec = MlaDecoder(w.batch, w.q_len, w.num_heads, device=dev)
+    shape = (w.batch, w.q_len, w.num_heads)
+    outs = []
+    dec.plan(sl)
+    for _ in range(3):  # one plan, three fused calls
+        o = torch.full(shape + (512,), float("nan"), dtype=torch.bfloat16, device=dev)
+        lse = torch.full(shape, float("nan"), dtype=torch.float32, device=dev)
+        dec.fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o=o, lse=lse)
+        outs.append((o.float().cpu().numpy(), lse.cpu().numpy()))
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    o_s = torch.full(shape + (512,), float("nan"), dtype=torch.bfloat16, device=dev)
+    l_s = torch.full(shape, float("nan"), dtype=torch.float32, device=dev)
+    dec.fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o=o_s, lse=l_s, flags=FLAG_SKIP_COMBINE)
+    mla_combine(dec.workspace, w.batch, w.q_len, w.num_heads, dec.n_sms, o_s, l_s)
+    torch.cuda.synchronize()
+    for o, l in outs:
+        np.testing.assert_array_equal(o, o_s.float().cpu().numpy())
+        np.testing.assert_array_equal(l, l_s.cpu().numpy())
+    assert_parity(outs[0][0], outs[0][1], *run_oracle(w), what=f"in-kernel merge h={heads}")
