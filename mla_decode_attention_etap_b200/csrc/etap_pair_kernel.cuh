@@ -147,9 +147,6 @@ __global__ void __launch_bounds__(320, 1)
     const int grp = cluster % p.groups;
     int32_t *status = p.ws + kHdrStatus;
 
-    // The schedule must come from a plan for this same grid (uniform in the whole cluster).
-    const bool plan_ok = p.ws[kHdrCtas] == p.ctas && p.ws[kHdrGroups] == p.groups && p.ws[kHdrBatch] == p.batch;
-
     auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * (uint32_t)i; };
     volatile WaitCtl *wc = reinterpret_cast<volatile WaitCtl *>(smem + C::OFF_MISC + 16);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
@@ -197,6 +194,15 @@ __global__ void __launch_bounds__(320, 1)
     cluster_sync();  // both CTAs' barriers are initialised before any remote arrive or st.async
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Launched as a programmatic dependent of the plan: everything above overlapped it; no
+    // global memory is read before the preceding grid has completed.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // A programmatic dependent launched next (the next plan) may be scheduled from now on; it
+    // waits for this grid to complete before touching memory.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // The schedule must come from a plan for this same grid (uniform in the whole cluster).
+    const bool plan_ok = p.ws[kHdrCtas] == p.ctas && p.ws[kHdrGroups] == p.groups && p.ws[kHdrBatch] == p.batch;
 
     const int32_t *ranges = p.ws + p.cta_ranges_off;
     const int32_t *tile_off = p.ws + p.tile_off_off;

@@ -106,13 +106,17 @@ cudaError_t launch_pair(const CUtensorMap &tm_q, const CUtensorMap &tm_kv, const
     cfg.blockDim = dim3(320, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_ALLOC;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // Programmatic dependent launch: the prologue (barriers, TMEM, descriptor prefetch)
+    // overlaps the preceding kernel; the kernel waits for it before any global read.
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, mla::etap_pair_kernel<C>, tm_q, tm_kv, tm_qr, tm_kvr, p);
 }
 
@@ -188,9 +192,21 @@ int mla_decode_plan(const int32_t *seqlens, int batch, int q_len, int num_heads,
     const mla::WsLayout lay = mla::ws_layout(batch, q_len, num_heads, num_sms);
     if (workspace_bytes < lay.total) return MLA_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    mla::plan_kernel<<<1, 256, 0, s>>>(seqlens, batch, lay.ctas, lay.groups, q_len * num_heads,
+    // Programmatic dependent launch: the plan is scheduled while the preceding kernel drains
+    // and waits for it to complete before its first global read.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, 1);
+    cfg.blockDim = dim3(mla::kPlanThreads, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, mla::plan_kernel, seqlens, batch, lay.ctas, lay.groups, q_len * num_heads,
                                        reinterpret_cast<int32_t *>(workspace), lay);
-    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "plan_kernel launch");
+    e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "plan_kernel launch");
     return MLA_OK;
 }

@@ -9,61 +9,104 @@
 
 namespace mla {
 
-// One CTA: tile prefix sums, per-CTA flattened ranges, per-sequence split info.
-// Writes the header (and clears the status word) so that the decode kernel can
-// check that it runs on a plan for its own grid.
-__global__ void plan_kernel(const int32_t *__restrict__ seqlens, int batch, int ctas, int groups, int ncols,
-                            int32_t *__restrict__ ws, WsLayout lay) {
+constexpr int kPlanThreads = 1024;
+
+// Exclusive prefix sum of one int64 per thread over the block; *total gets the block sum.
+__device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t *smem32, int64_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    int64_t incl = x;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    if (lane == 31) smem32[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int64_t w = lane < nwarps ? smem32[lane] : 0;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int64_t y = __shfl_up_sync(0xffffffffu, w, d);
+            if (lane >= d) w += y;
+        }
+        smem32[lane] = w;  // inclusive prefix of the warp sums
+    }
+    __syncthreads();
+    const int64_t base = warp > 0 ? smem32[warp - 1] : 0;
+    *total = smem32[nwarps - 1];
+    __syncthreads();  // smem32 is free for the next scan
+    return base + incl - x;
+}
+
+// One CTA: tile prefix sums, per-CTA flattened ranges, per-sequence split info, and
+// zeroed merge counters.  Writes the header (and clears the status word) so that the
+// decode kernel can check that it runs on a plan for its own grid.  kPlanThreads
+// threads; thread i owns the consecutive sequences [i*per, (i+1)*per).
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t *__restrict__ seqlens, int batch, int ctas,
+                                                            int groups, int ncols, int32_t *__restrict__ ws,
+                                                            WsLayout lay) {
+    // Launched as a programmatic dependent: nothing is read (seqlens may come from the
+    // preceding kernel) or written (that kernel may still read the workspace) before it
+    // completes.  Then the decode kernel may start its prologue: it waits for this grid in
+    // turn before reading the workspace.  Both are no-ops without programmatic launch.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ int64_t scan_smem[32];
     int32_t *tile_off = ws + lay.tile_off / 4;
     int32_t *ranges = ws + lay.cta_ranges / 4;
     int32_t *seq_info = ws + lay.seq_info / 4;
-    if (threadIdx.x == 0) {
-        int64_t acc = 0;
-        for (int b = 0; b < batch; ++b) {
-            tile_off[b] = (int32_t)acc;
-            acc += tiles_of(seqlens[b]);
-        }
-        tile_off[batch] = (int32_t)acc;
-    }
-    __syncthreads();
-    const int64_t total = tile_off[batch];
-    const int used = used_ctas(total, ctas);
-    for (int c = threadIdx.x; c < ctas; c += blockDim.x) {
-        ranges[2 * c] = (int32_t)cta_begin(total, used, c);
-        ranges[2 * c + 1] = (int32_t)cta_begin(total, used, c + 1);
-    }
     int32_t *counters = ws + lay.counters / 4;
-    for (int i = threadIdx.x; i < 2 * batch * groups; i += blockDim.x) counters[i] = 0;
-    for (int b = threadIdx.x; b < batch; b += blockDim.x) {
-        const int t0 = tile_off[b], t1 = tile_off[b + 1];
+    const int per = (batch + kPlanThreads - 1) / kPlanThreads;
+    const int b0 = min(batch, (int)threadIdx.x * per), b1 = min(batch, b0 + per);
+    // flattened tile offsets: exclusive prefix sum of tiles per sequence
+    int64_t mine = 0;
+    for (int b = b0; b < b1; ++b) mine += tiles_of(seqlens[b]);
+    int64_t total;
+    int64_t f = block_exclusive_scan(mine, scan_smem, &total);
+    const int used = used_ctas(total, ctas);
+    // splits per sequence (the consecutive CTAs its tiles fall on)
+    int64_t split_slots = 0;
+    for (int b = b0; b < b1; ++b) {
+        const int64_t t0 = f, t1 = f + tiles_of(seqlens[b]);
         int first = -1, nsplit = 0;
         if (t1 > t0) {
             first = cta_of(total, used, t0);
             nsplit = cta_of(total, used, t1 - 1) - first + 1;
         }
-        seq_info[4 * b + 0] = t1 - t0;
+        tile_off[b] = (int32_t)t0;
+        seq_info[4 * b + 0] = (int32_t)(t1 - t0);
         seq_info[4 * b + 1] = first;
         seq_info[4 * b + 2] = nsplit;
+        if (nsplit >= 2) split_slots += nsplit;
+        f = t1;
     }
-    __syncthreads();
+    // partial-output slots: exclusive prefix sum of the split counts of split sequences
+    int64_t slots;
+    int64_t sl = block_exclusive_scan(split_slots, scan_smem, &slots);
+    for (int b = b0; b < b1; ++b) {
+        seq_info[4 * b + 3] = (int32_t)sl;
+        if (seq_info[4 * b + 2] >= 2) sl += seq_info[4 * b + 2];
+    }
+    for (int c = threadIdx.x; c < ctas; c += kPlanThreads) {
+        ranges[2 * c] = (int32_t)cta_begin(total, used, c);
+        ranges[2 * c + 1] = (int32_t)cta_begin(total, used, c + 1);
+    }
+    for (int i = threadIdx.x; i < 2 * batch * groups; i += kPlanThreads) counters[i] = 0;
     if (threadIdx.x == 0) {
-        int slots = 0;
-        for (int b = 0; b < batch; ++b) {
-            seq_info[4 * b + 3] = slots;
-            if (seq_info[4 * b + 2] >= 2) slots += seq_info[4 * b + 2];
-        }
+        tile_off[batch] = (int32_t)total;
         ws[kHdrStatus] = 0;
         ws[kHdrCtas] = ctas;
         ws[kHdrGroups] = groups;
         ws[kHdrBatch] = batch;
         ws[kHdrTotalTiles] = (int32_t)total;
         ws[kHdrCols] = ncols;
-        ws[kHdrSlotsUsed] = slots;
+        ws[kHdrSlotsUsed] = (int32_t)slots;
         ws[kHdrSlotsMax] = lay.slots;
     }
 }
 
-// grid (ncols, batch), 128 threads: each thread merges 4 of the 512 output columns.
+// Stand-alone split merge: one CTA of 128 threads per (column, sequence), 4 latent rows
+// per thread.  Also writes O = 0, LSE = -inf for sequences without rows.
 __global__ void __launch_bounds__(128) combine_kernel(const int32_t *__restrict__ ws, const float *__restrict__ opart,
                                                       const float *__restrict__ lsepart, int ncols, WsLayout lay,
                                                       __nv_bfloat16 *__restrict__ o, float *__restrict__ lse) {

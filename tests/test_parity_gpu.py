@@ -240,3 +240,33 @@ def test_in_kernel_merge_matches_combine_and_resets_counters(heads):
         np.testing.assert_array_equal(o, o_s.float().cpu().numpy())
         np.testing.assert_array_equal(l, l_s.cpu().numpy())
     assert_parity(outs[0][0], outs[0][1], *run_oracle(w), what=f"in-kernel merge h={heads}")
+
+
+def _a256(x):
+    return (x + 255) & ~255
+
+
+@pytest.mark.parametrize("batch", [1, 7, 1024, 1500, 5000])
+def test_device_plan_matches_host_plan(batch):
+    """The block-scan plan kernel writes the same schedule as the host mirror (ranges, per-
+    sequence tiles / first unit / splits / slot offsets, tile offsets), for batches that give
+    each plan thread zero, one or several sequences, with empty sequences mixed in."""
+    from mla_decode_attention_etap_b200 import MlaDecoder, mla_decode_plan_host
+    rng = np.random.default_rng(batch)
+    lens = rng.integers(0, 3000, size=batch).astype(np.int32)
+    lens[rng.random(batch) < 0.2] = 0
+    dev = torch.device("cuda")
+    dec = MlaDecoder(batch, 1, 16, device=dev)
+    dec.plan(torch.tensor(lens, device=dev))
+    torch.cuda.synchronize()
+    ranges, info, nct, _ = mla_decode_plan_host(lens, 1, 16, dec.n_sms)
+    ws = dec.workspace.view(torch.int32).cpu().numpy()
+    off_ranges = _a256(4 * 64)
+    off_tile = off_ranges + _a256(4 * 2 * nct)
+    off_info = off_tile + _a256(4 * (batch + 1))
+    np.testing.assert_array_equal(ws[off_ranges // 4: off_ranges // 4 + 2 * nct].reshape(-1, 2), ranges)
+    np.testing.assert_array_equal(ws[off_info // 4: off_info // 4 + 4 * batch].reshape(-1, 4), info)
+    tiles = (lens.astype(np.int64) + 127) // 128
+    np.testing.assert_array_equal(ws[off_tile // 4: off_tile // 4 + batch + 1],
+                                  np.concatenate([[0], np.cumsum(tiles)]).astype(np.int32))
+    assert ws[0] == 0 and ws[1] == nct and ws[3] == batch and ws[4] == int(tiles.sum())
