@@ -44,7 +44,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_SOURCES = ["mla_decode_attention_etap_b200/csrc/etap_pair_kernel.cuh",
                   "mla_decode_attention_etap_b200/csrc/etap_common.cuh",
                   "mla_decode_attention_etap_b200/csrc/ptx_sm100.cuh",
-                  "mla_decode_attention_etap_b200/csrc/plan_core.h"]
+                  "mla_decode_attention_etap_b200/csrc/plan_core.h",
+                  "mla_decode_attention_etap_b200/csrc/merge.cuh"]
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "etap_pair_kernel_ncu.md")
 
 WORKLOADS = {

@@ -49,7 +49,7 @@ struct PairCfg {
     static constexpr int PAIRS = 2;                                    // V pairs of a tile in one CTA
     static constexpr int EARLY = (NV - PAIRS) < PAIRS ? (NV - PAIRS) : PAIRS;  // pairs of tile k+1 free of tile k
     static constexpr int XS = CH > 2 ? CH : 2;                         // exchange slots (8 KB each)
-    static constexpr int PREFETCH = 2;                                 // tiles the L2 prefetch runs ahead of the loads
+    static constexpr int PREFETCH = 1;                                 // tiles the L2 prefetch runs ahead of the loads
     static constexpr uint32_t CHUNK = 16384;                           // 128 rows x 64 bf16, 128B swizzle
     static constexpr uint32_t HALF = 8192;                             // 64 rows of a chunk = one TMA box
     static constexpr uint32_t V_SLOT = 2 * CHUNK;
