@@ -18,6 +18,12 @@ constexpr uint64_t kWaitLimitNs = 4000000000ull;     // default bound of every w
 constexpr uint64_t kTestWaitLimitNs = 100000000ull;  // bound used by the expired-wait test hook
 constexpr uint64_t kDrainLimitNs = 200000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p = 2^(x - m) stays <= 256
+// When the running maximum of a column moves, it is set this far (log2 units) above the tile's
+// maximum, so that later tiles rarely cross the threshold again (each crossing costs a cross-warp
+// reduction and an O^T rescale).  p then starts at 2^-24 for the row of the maximum: fp32 and the
+// bf16 hi + lo split keep their relative precision there, and only rows more than ~100 octaves
+// below the maximum underflow to 0, as they would in any fp32 softmax.
+constexpr float kRescaleHeadroom = 24.0f;
 
 // Per-CTA wait control in shared memory: the abort flag every role polls and
 // the bound after which a wait gives up.

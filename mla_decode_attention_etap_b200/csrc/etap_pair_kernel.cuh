@@ -681,10 +681,10 @@ __global__ void __launch_bounds__(320, 1)
                                 for (int u = 0; u < 4; ++u) {
                                     const int n = n4 + u, li = 8 * ch + n;
                                     if (first) {
-                                        m[li] = mt4[u];
+                                        m[li] = mt4[u] + kRescaleHeadroom;
                                     } else if (mt4[u] > m[li] + kRescaleThreshold) {
-                                        alpha[ch][n] = fast_exp2(m[li] - mt4[u]);
-                                        m[li] = mt4[u];
+                                        alpha[ch][n] = fast_exp2(m[li] - (mt4[u] + kRescaleHeadroom));
+                                        m[li] = mt4[u] + kRescaleHeadroom;
                                         rescale = true;
                                     }
                                 }
