@@ -117,11 +117,26 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+def code_only(text: str) -> str:
+    """Source text without // comments and blank lines: what the compiler sees, for the hash."""
+    out = []
+    for line in text.splitlines():
+        code = line.split("//", 1)[0].rstrip()
+        if code.strip():
+            out.append(code)
+    return "\n".join(out)
+
+
+def kernel_source_hash(read=None) -> str:
+    """Hash of the decode kernel's sources (code only, so that comment edits keep a profile valid)."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        if read is None:
+            with open(os.path.join(ROOT, rel)) as f:
+                text = f.read()
+        else:
+            text = read(rel)
+        h.update(code_only(text).encode())
     return h.hexdigest()[:16]
 
 

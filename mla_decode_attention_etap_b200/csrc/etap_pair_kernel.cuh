@@ -13,18 +13,21 @@
 //     A 128-row tile then needs 72 KB of shared memory per CTA instead of
 //     144 KB, so each CTA's ring keeps ~2.5 tiles in flight and
 //     the loads of tile k+1 overlap the softmax and the second contraction of
-//     tile k.  Each CTA computes a partial S^T over its own columns; the 128
-//     softmax threads send their rows of it to the peer CTA (st.async into the
-//     peer's shared memory, counted on the peer's mbarrier) and add the peer's
-//     rows, so both CTAs hold the same S^T (fp32 addition commutes), run the
-//     same softmax and each accumulates O^T for its own 256 value columns.
+//     tile k.  Each CTA computes a partial S^T over its own columns; the 256
+//     softmax threads send their part of it to the peer CTA (st.async into the
+//     peer's shared memory, counted on the peer's per-warp mbarriers) and add
+//     the peer's part, so both CTAs hold the same S^T (fp32 addition commutes),
+//     run the same softmax and each accumulates O^T for its own 256 value columns.
 //   * warp 0: TMA producer (Q once per segment, KV tiles into 32 KB slots of
-//     two 64-column chunks plus an 8 KB slot for the 32 rope columns; tail
-//     rows zeroed);
-//   * warp 1 lane 0: tcgen05.mma issuer, S^T of tile k+1 before O^T of tile k;
-//   * warps 2..9: one TMEM lane (= one KV row) and half of the columns per
-//     thread; the column softmax reduces ACROSS threads; P^T goes to shared
-//     memory as bf16 hi | lo.
+//     two 64-column chunks plus 8 KB slots for the 32 rope columns; tail rows
+//     zeroed; L2 prefetch one tile ahead);
+//   * warp 1 lane 0: tcgen05.mma issuer, an event loop over the score MMAs of
+//     the next tile (in stages, as their operands land) and O^T of the oldest
+//     tile whose P^T is ready;
+//   * warps 2..9: two warps per TMEM lane quadrant, one KV row and half of the
+//     columns per thread; the column softmax reduces ACROSS threads; P^T goes
+//     to shared memory as bf16 hi | lo; at the end of a split the last CTA of
+//     a sequence merges the split partials (log-sum-exp).
 //
 // Every wait is bounded; see etap_common.cuh.
 #pragma once
