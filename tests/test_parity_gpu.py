@@ -270,3 +270,13 @@ def test_device_plan_matches_host_plan(batch):
     np.testing.assert_array_equal(ws[off_tile // 4: off_tile // 4 + batch + 1],
                                   np.concatenate([[0], np.cumsum(tiles)]).astype(np.int32))
     assert ws[0] == 0 and ws[1] == nct and ws[3] == batch and ws[4] == int(tiles.sum())
+
+
+@pytest.mark.parametrize("heads,q_len,causal", [(64, 1, False), (128, 2, False), (32, 4, True), (16, 8, True),
+                                                (128, 8, True)])
+def test_many_column_groups(heads, q_len, causal):
+    """h*q_len from 64 to 1024 columns: 2..32 column groups of 32 (one cluster each per unit)."""
+    w = W.make_workload(2, heads, [700, 130], q_len=q_len, causal=causal, seed=heads + q_len, paged=heads >= 128)
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"h={heads} q={q_len}")
