@@ -52,6 +52,10 @@ struct PairCfg {
     static constexpr int PAIRS = 2;                                    // V pairs of a tile in one CTA
     static constexpr int EARLY = (NV - PAIRS) < PAIRS ? (NV - PAIRS) : PAIRS;  // pairs of tile k+1 free of tile k
     static constexpr int XS = CH > 2 ? CH : 2;                         // exchange slots (8 KB each)
+    // One column chunk per thread (h*q_len <= 16): the softmax warps issue step 3 themselves, right
+    // after the barrier that ends the tile, instead of handing P^T to the MMA warp (its polling and
+    // the score MMAs it may be issuing would delay it); the issuing warp has a tile's time to spare.
+    static constexpr bool PV_BY_SOFTMAX = CH == 1;
     static constexpr int PREFETCH = 1;                                 // tiles the L2 prefetch runs ahead of the loads
     static constexpr uint32_t CHUNK = 16384;                           // 128 rows x 64 bf16, 128B swizzle
     static constexpr uint32_t HALF = 8192;                             // 64 rows of a chunk = one TMA box
@@ -111,7 +115,8 @@ struct PairBars {
     static constexpr int PEMPTY = PFULL + C::PB;
     static constexpr int TAIL = PEMPTY + C::PB;
     static constexpr int FINAL = TAIL + 1;
-    static constexpr int RED = FINAL + 1;
+    static constexpr int SFIN = FINAL + 1;  // drain of the step-3 MMAs a softmax thread issued
+    static constexpr int RED = SFIN + 1;
     static constexpr int REDL = RED + 1;
     // Exchange barriers are per softmax warp: warp w only needs (and only frees) the partial
     // scores of the peer's warp w (same rows, same columns), and one barrier per warp keeps the
@@ -175,6 +180,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         mbar_init(bar(BR::TAIL), 1);
         mbar_init(bar(BR::FINAL), 1);
+        mbar_init(bar(BR::SFIN), 1);
         mbar_init(bar(BR::RED), 4);
         mbar_init(bar(BR::REDL), 4);
         for (int i = 0; i < 8 * C::XS; ++i) mbar_init(bar(BR::XFULL + i), 1);
@@ -197,6 +203,28 @@ __global__ void __launch_bounds__(320, 1)
     cluster_sync();  // both CTAs' barriers are initialised before any remote arrive or st.async
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Step 3 of tile kk: O^T (+)= V^T P^T for both V pairs of this CTA; frees each V slot and then
+    // the P^T buffer as the MMAs complete.
+    auto issue_pv = [&](int kk, bool first) {
+        const int pb = kk % C::PB;
+        const uint32_t p_base = sbase + C::OFF_P + pb * C::P_BUF;
+        for (int i = 0; i < C::PAIRS; ++i) {
+            const int g2 = C::PAIRS * kk + i;
+            const int vs = g2 % C::NV;
+            const uint32_t v_base = sbase + C::OFF_V + vs * C::V_SLOT;
+            const uint32_t d_o = tmem + C::O_COL + i * C::NP;
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                // A = V^T: M = 128 latent columns (two chunks CHUNK apart), K = 16 KV rows (MN-major)
+                const uint64_t a = smem_desc(v_base + 2048u * s, C::CHUNK, 1024, kSwizzle128B);
+                // B = [P_hi | P_lo]^T: K = 16 KV rows, N = NP columns (MN-major)
+                const uint64_t bp = smem_desc(p_base + 16u * C::P_PITCH * s, C::P_ATOM, 8 * C::P_PITCH, C::P_SWIZZLE);
+                umma_bf16(d_o, a, bp, C::IDESC_PV, (first && s == 0) ? 0u : 1u);
+            }
+            umma_commit(bar(BR::VEMPTY + vs));
+        }
+        umma_commit(bar(BR::PEMPTY + pb));
+    };
     // Launched as a programmatic dependent of the plan: everything above overlapped it; no
     // global memory is read before the preceding grid has completed.
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -405,32 +433,13 @@ __global__ void __launch_bounds__(320, 1)
             int kq = 0, kp = 0, seg_q = 0;
             int qstage = 0;  // scores of tile kq: 0 = rope columns next, 1 + i = V pair i next
             uint64_t t_last = global_timer_ns();
-            while (pc.valid) {
+            while (C::PV_BY_SOFTMAX ? qc.valid : pc.valid) {
                 bool progressed = false;
                 // step 3 first when its P^T is ready: it frees V slots for later tiles
-                if (kp < kq) {
-                    const int pb = kp % C::PB;
-                    if (mbar_test_wait(bar(BR::PFULL + pb), (kp / C::PB) & 1)) {
+                if constexpr (!C::PV_BY_SOFTMAX) {
+                    if (kp < kq && mbar_test_wait(bar(BR::PFULL + kp % C::PB), (kp / C::PB) & 1)) {
                         tc_fence_after();
-                        const bool first = pc.first();
-                        const uint32_t p_base = sbase + C::OFF_P + pb * C::P_BUF;
-                        for (int i = 0; i < C::PAIRS; ++i) {
-                            const int g2 = C::PAIRS * kp + i;
-                            const int vs = g2 % C::NV;
-                            const uint32_t v_base = sbase + C::OFF_V + vs * C::V_SLOT;
-                            const uint32_t d_o = tmem + C::O_COL + i * C::NP;
-#pragma unroll
-                            for (int s = 0; s < 8; ++s) {
-                                // A = V^T: M = 128 latent columns (two chunks CHUNK apart), K = 16 KV rows (MN-major)
-                                const uint64_t a = smem_desc(v_base + 2048u * s, C::CHUNK, 1024, kSwizzle128B);
-                                // B = [P_hi | P_lo]^T: K = 16 KV rows, N = NP columns (MN-major)
-                                const uint64_t bp = smem_desc(p_base + 16u * C::P_PITCH * s, C::P_ATOM,
-                                                              8 * C::P_PITCH, C::P_SWIZZLE);
-                                umma_bf16(d_o, a, bp, C::IDESC_PV, (first && s == 0) ? 0u : 1u);
-                            }
-                            umma_commit(bar(BR::VEMPTY + vs));
-                        }
-                        umma_commit(bar(BR::PEMPTY + pb));
+                        issue_pv(kp, pc.first());
                         pc.advance(tile_off);
                         ++kp;
                         progressed = true;
@@ -514,7 +523,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t xfull_remote = map_to_rank(bar(BR::XFULL + sw), peer);
         const uint32_t xfree_remote = map_to_rank(bar(BR::XFREE + sw), peer);
         const int k_total = (int)(fe - fb);
-        bool ok = true, stop = false;
+        bool ok = true, stop = false, pv_issued = false;
         // Exchange slots hold 128 rows x 16 fp32; this thread's 8 values are 16-byte chunks 2*half, 2*half+1.
         auto x_off = [&](int j) -> uint32_t { return swz_off(row, 2 * half + j, 64, 3); };
         // CH > 1: whole-tile exchange, one tile ahead.  Our partial S^T of tile kk goes to the
@@ -760,8 +769,18 @@ __global__ void __launch_bounds__(320, 1)
                     if (rescale_any) tmem_wait_st();
                     fence_proxy_async_smem();
                     tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(BR::PFULL + pb));
+                    if constexpr (C::PV_BY_SOFTMAX) {
+                        // every P^T row written and every O^T rescale done: one thread issues step 3
+                        named_bar_sync(SMX, NSM);
+                        if (warp == 2 && lane == 0) {
+                            tc_fence_after();
+                            issue_pv(k, first);
+                            pv_issued = true;
+                        }
+                    } else {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(BR::PFULL + pb));
+                    }
                     if constexpr (C::CH > 1) {
                         if (k + 1 < k_total && !sent_next) send_tile(k + 1);
                     }
@@ -927,6 +946,11 @@ __global__ void __launch_bounds__(320, 1)
             }
         }
         if (stop || !ok) wc->abort = 1;
+        if (pv_issued) {
+            // the step-3 MMAs this thread issued complete before TMEM is released
+            umma_commit(bar(BR::SFIN));
+            drain_phase(bar(BR::SFIN), 0);
+        }
         __syncwarp();
     }
 
