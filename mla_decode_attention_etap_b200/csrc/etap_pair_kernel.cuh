@@ -22,8 +22,9 @@
 //     two 64-column chunks plus 8 KB slots for the 32 rope columns; tail rows
 //     zeroed; L2 prefetch one tile ahead);
 //   * warp 1 lane 0: tcgen05.mma issuer, an event loop over the score MMAs of
-//     the next tile (in stages, as their operands land) and O^T of the oldest
-//     tile whose P^T is ready;
+//     the next tile (in stages, as their operands land) and, for 32-column
+//     groups, O^T of the oldest tile whose P^T is ready (for 16 columns one
+//     softmax thread issues O^T right after the barrier that ends the tile);
 //   * warps 2..9: two warps per TMEM lane quadrant, one KV row and half of the
 //     columns per thread; the column softmax reduces ACROSS threads; P^T goes
 //     to shared memory as bf16 hi | lo; at the end of a split the last CTA of
@@ -414,9 +415,10 @@ __global__ void __launch_bounds__(320, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         // An event loop: step 1 of the next tile goes as soon as its KV and Q are
-        // in shared memory, step 3 of the oldest pending tile as soon as its P^T
-        // is; "S^T ready" is committed right after the scores' MMAs, so the
-        // softmax of tile k overlaps step 3 of tile k-1 on the tensor pipe.
+        // in shared memory, step 3 of the oldest pending tile (unless the softmax
+        // warps issue it) as soon as its P^T is; "S^T ready" is committed right
+        // after the scores' MMAs, so the softmax of tile k overlaps step 3 of
+        // tile k-1 on the tensor pipe.
         if (lane == 0 && fb < fe) {
             const uint32_t q_base = sbase + C::OFF_Q;
             auto qk_chunk = [&](uint32_t d_s, uint32_t a_base, int qchunk, bool init) {
