@@ -20,6 +20,13 @@
  * (the q_len new tokens are the last q_len cache rows).  A column with no
  * visible row gives O = 0 and LSE = -inf.
  *
+ * Ragged multi-token decode (a different number of new tokens per sequence,
+ * q_lens[b] <= q_len; the pages decode one token per forward and name more
+ * as a limitation, "Discussion"): token t of sequence b is a real query iff
+ * t < q_lens[b], and then it sees j <= L_b - q_lens[b] + t when causal (its
+ * q_lens[b] new tokens are the last q_lens[b] cache rows) or j < L_b; padding
+ * tokens t >= q_lens[b] see no row (O = 0, LSE = -inf).
+ *
  * Inputs are bf16 bit patterns (uint16), widened exactly to fp64.  All
  * arithmetic is fp64.  Paged caches ([num_blocks, page, 576]) are resolved
  * through the block table; contiguous caches are [B, kv_rows, 576].
@@ -54,6 +61,20 @@ static int visible_rows(int L, int q_len, int t, int causal)
     return vis < 0 ? 0 : vis;
 }
 
+/* Visible rows of token t of sequence b: uniform q_len, or ragged when q_lens != NULL. */
+static int token_visible_rows(int L, int q_len, const int32_t *q_lens, int b, int t, int causal)
+{
+    if (!q_lens) return visible_rows(L, q_len, t, causal);
+    int qb = q_lens[b];
+    if (t >= qb) return 0;
+    return visible_rows(L, qb, t, causal);
+}
+
+static int decode_standard(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
+                           const int32_t *q_lens, const int32_t *block_table, int B, int q_len, int h,
+                           int d_qk, int d_v, int kv_rows, int max_blocks, int page, double scale,
+                           int causal, double *o, double *lse);
+
 /*
  * Standard form: S = Q K^T, P = softmax(S) over the KV axis, O = P V.
  * q: [B, q_len, h, d_qk]; o: [B, q_len, h, d_v]; lse: [B, q_len, h].
@@ -64,6 +85,25 @@ int oracle_mla_decode(const uint16_t *q, const uint16_t *kv, const int32_t *seql
                       int kv_rows, int max_blocks, int page, double scale, int causal,
                       double *o, double *lse)
 {
+    return decode_standard(q, kv, seqlens, NULL, block_table, B, q_len, h, d_qk, d_v, kv_rows,
+                           max_blocks, page, scale, causal, o, lse);
+}
+
+/* The same with q_lens[b] real query tokens in sequence b (0 <= q_lens[b] <= q_len). */
+int oracle_mla_decode_ragged(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
+                             const int32_t *q_lens, const int32_t *block_table, int B, int q_len,
+                             int h, int d_qk, int d_v, int kv_rows, int max_blocks, int page,
+                             double scale, int causal, double *o, double *lse)
+{
+    return decode_standard(q, kv, seqlens, q_lens, block_table, B, q_len, h, d_qk, d_v, kv_rows,
+                           max_blocks, page, scale, causal, o, lse);
+}
+
+static int decode_standard(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
+                           const int32_t *q_lens, const int32_t *block_table, int B, int q_len, int h,
+                           int d_qk, int d_v, int kv_rows, int max_blocks, int page, double scale,
+                           int causal, double *o, double *lse)
+{
     int rows = B * q_len * h;
     int failed = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : failed)
@@ -71,7 +111,7 @@ int oracle_mla_decode(const uint16_t *q, const uint16_t *kv, const int32_t *seql
         int b = r / (q_len * h);
         int t = (r / h) % q_len;
         int L = seqlens[b];
-        int vis = visible_rows(L, q_len, t, causal);
+        int vis = token_visible_rows(L, q_len, q_lens, b, t, causal);
         const uint16_t *qr = q + (int64_t)r * d_qk;
         double *orow = o + (int64_t)r * d_v;
         double qd[1024];

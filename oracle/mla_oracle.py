@@ -57,6 +57,8 @@ def _load():
             fn = getattr(lib, name)
             fn.argtypes = args
             fn.restype = ctypes.c_int
+        lib.oracle_mla_decode_ragged.argtypes = args[:3] + [ctypes.c_void_p] + args[3:]
+        lib.oracle_mla_decode_ragged.restype = ctypes.c_int
         lib.oracle_lse_merge.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_lse_merge.restype = None
@@ -68,7 +70,7 @@ def _ptr(a: Optional[np.ndarray]):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
-def _call(name, q_bits, kv_bits, seqlens, block_table, scale, causal, threads=None):
+def _call(name, q_bits, kv_bits, seqlens, block_table, scale, causal, threads=None, q_lens=None):
     q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
     kv_bits = np.ascontiguousarray(kv_bits, dtype=np.uint16)
     seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
@@ -83,17 +85,27 @@ def _call(name, q_bits, kv_bits, seqlens, block_table, scale, causal, threads=No
     lse = np.zeros((B, q_len, h), dtype=np.float64)
     if threads is not None:
         os.environ["OMP_NUM_THREADS"] = str(threads)
-    rc = getattr(_load(), name)(_ptr(q_bits), _ptr(kv_bits), _ptr(seqlens), _ptr(block_table),
-                                B, q_len, h, D_QK, D_V, kv_rows, max_blocks, page,
-                                float(scale), int(bool(causal)), _ptr(o), _ptr(lse))
+    if q_lens is None:
+        rc = getattr(_load(), name)(_ptr(q_bits), _ptr(kv_bits), _ptr(seqlens), _ptr(block_table),
+                                    B, q_len, h, D_QK, D_V, kv_rows, max_blocks, page,
+                                    float(scale), int(bool(causal)), _ptr(o), _ptr(lse))
+    else:
+        q_lens = np.ascontiguousarray(q_lens, dtype=np.int32)
+        assert q_lens.shape == (B,) and q_lens.min() >= 0 and q_lens.max() <= q_len
+        rc = _load().oracle_mla_decode_ragged(_ptr(q_bits), _ptr(kv_bits), _ptr(seqlens), _ptr(q_lens),
+                                              _ptr(block_table), B, q_len, h, D_QK, D_V, kv_rows, max_blocks,
+                                              page, float(scale), int(bool(causal)), _ptr(o), _ptr(lse))
     if rc != 0:
         raise MemoryError(f"{name} failed ({rc})")
     return o, lse
 
 
-def mla_decode(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.0, causal=False):
-    """Standard-form oracle.  Returns (O fp64 [B,q,h,512], LSE fp64 [B,q,h])."""
-    return _call("oracle_mla_decode", q_bits, kv_bits, seqlens, block_table, scale, causal)
+def mla_decode(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.0, causal=False, q_lens=None):
+    """Standard-form oracle.  Returns (O fp64 [B,q,h,512], LSE fp64 [B,q,h]).
+
+    ``q_lens`` (optional, [B]): ragged multi-token decode, q_lens[b] real query tokens in
+    sequence b (the rest of the q_len positions are padding: O = 0, LSE = -inf)."""
+    return _call("oracle_mla_decode", q_bits, kv_bits, seqlens, block_table, scale, causal, q_lens=q_lens)
 
 
 def mla_decode_etap(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.0, causal=False):
@@ -126,7 +138,7 @@ def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return rounded.astype(np.uint16)
 
 
-def mla_decode_numpy(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.0, causal=False):
+def mla_decode_numpy(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.0, causal=False, q_lens=None):
     """Second, independent fp64 implementation of the standard form with numpy matmuls."""
     q = bf16_bits_to_f64(q_bits)
     kv = bf16_bits_to_f64(kv_bits)
@@ -141,8 +153,12 @@ def mla_decode_numpy(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.
             rows = kv[np.asarray(block_table[b, :nb], dtype=np.int64)].reshape(nb * page, D_QK)[:L]
         else:
             rows = kv[b, :L]
+        qb = q_len if q_lens is None else int(q_lens[b])
         for t in range(q_len):
-            vis = max(L - q_len + t + 1, 0) if causal else L
+            if t >= qb:
+                vis = 0                                   # padding token of a ragged batch
+            else:
+                vis = max(L - qb + t + 1, 0) if causal else L
             if vis == 0:
                 lse[b, t] = -math.inf
                 continue

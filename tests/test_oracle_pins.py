@@ -374,3 +374,55 @@ def test_empty_sequence_and_fully_masked_columns():
 def test_lse_merge_all_empty():
     o, lse = om.lse_merge(np.zeros((3, D_V)), np.array([-math.inf] * 3))
     assert lse == -math.inf and np.all(o == 0)
+
+
+# ---------------------------------------------------------------- ragged multi-token decode
+# q_lens[b] real query tokens in sequence b; the q_lens[b] new tokens are the last q_lens[b] cache
+# rows.  Pinned against the uniform form (itself pinned above): sequence b of a ragged batch is
+# the uniform decode of that sequence alone with q_len = q_lens[b], and padding tokens see nothing.
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("ragged", ["c", "numpy"])
+def test_ragged_equals_each_sequence_decoded_alone(causal, ragged):
+    rng = np.random.default_rng(30)
+    sl = np.array([300, 5, 129, 2], np.int32)
+    q_lens = np.array([1, 4, 2, 3], np.int32)
+    q = rand_bits(rng, (4, 4, 3, D_QK))
+    kv = rand_bits(rng, (4, 300, D_QK))
+    fn = om.mla_decode if ragged == "c" else om.mla_decode_numpy
+    o, lse = fn(q, kv, sl, None, SCALE, causal, q_lens=q_lens)
+    for b in range(4):
+        qb = int(q_lens[b])
+        o1, l1 = om.mla_decode(q[b:b + 1, :qb], kv[b:b + 1], sl[b:b + 1], None, SCALE, causal)
+        np.testing.assert_allclose(o[b, :qb], o1[0], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[b, :qb], l1[0], rtol=0, atol=1e-13)
+        assert np.all(o[b, qb:] == 0) and np.all(np.isneginf(lse[b, qb:]))
+
+
+def test_ragged_with_full_lengths_is_the_uniform_decode():
+    rng = np.random.default_rng(31)
+    sl = np.array([70, 130], np.int32)
+    q = rand_bits(rng, (2, 3, 2, D_QK))
+    kv = rand_bits(rng, (2, 130, D_QK))
+    for causal in (False, True):
+        ref = om.mla_decode(q, kv, sl, None, SCALE, causal)
+        got = om.mla_decode(q, kv, sl, None, SCALE, causal, q_lens=np.array([3, 3], np.int32))
+        np.testing.assert_array_equal(got[0], ref[0])
+        np.testing.assert_array_equal(got[1], ref[1])
+
+
+def test_ragged_causal_offset_uses_the_sequence_own_token_count():
+    """Token 0 of a sequence with 2 new tokens sees L-1 rows (not L-q_max+1): with q_max = 4 and
+    L = 6 a wrong offset would give it 3 rows; check the visible count through a one-hot V."""
+    L, h = 6, 1
+    q = np.zeros((1, 4, h, D_QK), np.uint16)                   # Q = 0: equal scores, O = mean of visible V
+    kv = np.zeros((1, L, D_QK), np.float64)
+    kv[0, :, 0] = 1.0                                          # every visible row contributes 1 to O[0]
+    kv[0, :, 1] = np.arange(L)                                 # O[1] = mean row index of the visible rows
+    kvb = om.f64_to_bf16_bits(kv)
+    o, lse = om.mla_decode(q, kvb, np.array([L], np.int32), None, SCALE, True, q_lens=np.array([2], np.int32))
+    # token 0 sees rows 0..4 (mean 2.0, LSE ln 5), token 1 sees rows 0..5 (mean 2.5, LSE ln 6)
+    np.testing.assert_allclose(o[0, 0, 0, 1], 2.0, atol=1e-12)
+    np.testing.assert_allclose(o[0, 1, 0, 1], 2.5, atol=1e-12)
+    np.testing.assert_allclose(lse[0, :2, 0], [math.log(5), math.log(6)], atol=1e-12)
+    assert np.all(np.isneginf(lse[0, 2:]))
