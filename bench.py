@@ -57,6 +57,7 @@ WORKLOADS = {
     "b64_h16_paged": dict(kind="b64_paged"),
     "b32_h128_paged": dict(kind="b32_h128"),
     "b16_h16_q4_causal": dict(kind="q4_causal"),
+    "b16_h16_ragged_q4_causal": dict(kind="ragged_q4_causal"),
 }
 
 
@@ -103,6 +104,9 @@ def make_workload(name: str, rank: int, device):
     if kind == "q4_causal":
         return (W.workload_b16_h16_q4_causal(seed=seed, device=device),
                 "mla_decode_b16_h16_q4_causal_L32768_spikes5pct_x8")
+    if kind == "ragged_q4_causal":
+        return (W.workload_b16_h16_ragged_q4_causal(seed=seed, device=device),
+                "mla_decode_b16_h16_ragged_q1to4_causal_L32768_spikes5pct_x8")
     w = W.make_workload(spec["batch"], spec["heads"], [spec["seqlen"]] * spec["batch"], seed=seed, device=device)
     return w, f"mla_decode_b{spec['batch']}_h{spec['heads']}_q1_L{spec['seqlen']}_contiguous"
 
@@ -217,6 +221,13 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CPU baseline (oracle)
+def W_flops(seqlens, w, q_lens=None) -> int:
+    """Algorithmic flops of the listed sequences of workload ``w`` (q_lens: their token counts)."""
+    from mla_decode_attention_etap_b200 import workloads as W
+    return W.algorithmic_flops(seqlens, w.q_len, w.num_heads, w.causal,
+                               None if q_lens is None else [int(x) for x in q_lens])
+
+
 def oracle_baseline(w, target_s: float = 12.0):
     """Time the fp64 oracle on whole sequences of the workload until ~target_s of CPU work."""
     import numpy as np
@@ -234,12 +245,12 @@ def oracle_baseline(w, target_s: float = 12.0):
         rows = w.kv_rows(b).cpu()
         kv = bf16_bits(rows.reshape(1, L, 576))
         q = bf16_bits(w.q[b:b + 1].cpu())
+        ql = None if w.q_lens is None else w.q_lens[b:b + 1].numpy()
         t0 = time.perf_counter()
-        om.mla_decode(q, kv, np.array([L], np.int32), None, w.softmax_scale, w.causal)
+        om.mla_decode(q, kv, np.array([L], np.int32), None, w.softmax_scale, w.causal, q_lens=ql)
         t_total += time.perf_counter() - t0
         done_bytes += L * 1152
-        vis = sum(max((L - w.q_len + t + 1) if w.causal else L, 0) for t in range(w.q_len))
-        done_flops += vis * w.num_heads * 2 * 1088
+        done_flops += W_flops([L], w, ql)
         seqs.append(b)
         if t_total >= target_s:
             break
@@ -269,19 +280,19 @@ def run_reference(args):
     kv = bf16_bits(w.kv_rows(b)[:L].cpu().reshape(1, L, 576))
     q = bf16_bits(w.q[b:b + 1].cpu())
     sl = np.array([L], np.int32)
+    ql = None if w.q_lens is None else w.q_lens[b:b + 1].numpy()
     for _ in range(args.warmup):
-        om.mla_decode(q, kv, sl, None, w.softmax_scale, w.causal)
+        om.mla_decode(q, kv, sl, None, w.softmax_scale, w.causal, q_lens=ql)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        om.mla_decode(q, kv, sl, None, w.softmax_scale, w.causal)
+        om.mla_decode(q, kv, sl, None, w.softmax_scale, w.causal, q_lens=ql)
     dt = (time.perf_counter() - t0) / args.steps
     value = L * 1152 / dt / 1e12
-    vis = sum(max((L - w.q_len + t + 1) if w.causal else L, 0) for t in range(w.q_len))
     sample = f"sequence 0, first {L} cache rows, all {w.num_heads} heads x {w.q_len} token(s), per step"
     line = {"metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "tflops": vis * w.num_heads * 2 * 1088 / dt / 1e12,
+            "tflops": W_flops([L], w, ql) / dt / 1e12,
             "config": {"workload": wname, "reference_sample": sample},
             "cpu_baseline": {"value": value, "unit": "TB/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -312,7 +323,8 @@ def run_ours(args):
     lse = torch.empty(B, q_len, h, dtype=torch.float32, device=dev)
     seqlens = [int(x) for x in w.seqlens]
     kv_bytes = W.algorithmic_kv_bytes(seqlens)
-    flops = W.algorithmic_flops(seqlens, q_len, h, w.causal)
+    q_lens = w.q_lens.to(dev) if w.q_lens is not None else None
+    flops = W.algorithmic_flops(seqlens, q_len, h, w.causal, None if w.q_lens is None else w.q_lens.tolist())
     stream = torch.cuda.current_stream()
 
     n_events = args.steps
@@ -323,7 +335,8 @@ def run_ours(args):
         if i is not None:
             ev[i][0].record(stream)
         # the decode kernel merges the split-KV partials itself (no combine launch)
-        mla.mla_decode_fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o, lse, dec.workspace, dec.n_sms, 0)
+        mla.mla_decode_fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o, lse, dec.workspace, dec.n_sms, 0,
+                           q_lens=q_lens)
         if i is not None:
             ev[i][1].record(stream)
 
@@ -366,7 +379,10 @@ def run_ours(args):
     hl = torch.empty_like(lse, device="cpu").pin_memory()
     dq, dkv, dsl = torch.empty_like(q), torch.empty_like(kv), torch.empty_like(sl)
     dbt = torch.empty_like(bt) if bt is not None else None
-    h2d = hq.numel() * 2 + hkv.numel() * 2 + hsl.numel() * 4 + (hbt.numel() * 4 if hbt is not None else 0)
+    hql = w.q_lens.clone().pin_memory() if w.q_lens is not None else None
+    dql = torch.empty_like(q_lens) if q_lens is not None else None
+    h2d = (hq.numel() * 2 + hkv.numel() * 2 + hsl.numel() * 4 + (hbt.numel() * 4 if hbt is not None else 0)
+           + (hql.numel() * 4 if hql is not None else 0))
     d2h = ho.numel() * 2 + hl.numel() * 4
 
     def e2e_step():
@@ -375,8 +391,11 @@ def run_ours(args):
         dsl.copy_(hsl, non_blocking=True)
         if dbt is not None:
             dbt.copy_(hbt, non_blocking=True)
+        if dql is not None:
+            dql.copy_(hql, non_blocking=True)
         dec.plan(dsl)
-        mla.mla_decode_fwd(dq, dkv, dsl, dbt, w.softmax_scale, w.causal, o, lse, dec.workspace, dec.n_sms, 0)
+        mla.mla_decode_fwd(dq, dkv, dsl, dbt, w.softmax_scale, w.causal, o, lse, dec.workspace, dec.n_sms, 0,
+                           q_lens=dql)
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
@@ -425,6 +444,7 @@ def run_ours(args):
             "data": "synthetic",
             "tflops": weak_scaling_value(flops, world, step_s_max) / 1e12,
             "config": {"workload": wname, "batch_per_gpu": B, "heads": h, "q_len": q_len,
+                       "q_lens": None if w.q_lens is None else w.q_lens.tolist(),
                        "seqlens": (seqlens[0] if len(set(seqlens)) == 1 else
                                    f"{min(seqlens)}..{max(seqlens)} (mean {sum(seqlens) / len(seqlens):.0f})"),
                        "d_qk": 576, "d_v": 512, "kv_layout": "paged64" if bt is not None else "contiguous",

@@ -130,6 +130,26 @@ MLA_API int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens
                    void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream);
 
 /*
+ * Ragged multi-token decode: as mla_decode_fwd, with a different number of new
+ * query tokens per sequence.  The pages decode one token per forward and name
+ * more as a limitation (FlashMLA-ETAP technical summary, "Discussion"); this is
+ * the speculative-verify shape with per-sequence draft lengths.
+ *   q_lens   int32 [batch], device, 0 <= q_lens[b] <= q_len, or NULL (all q_len).
+ *            Sequence b's real query tokens are rows t < q_lens[b] of its q_len
+ *            query rows; they are the last q_lens[b] cache rows, so with causal = 1
+ *            token t sees cache rows j <= L_b - q_lens[b] + t (else j < L_b).
+ *            Rows t >= q_lens[b] are padding: O = 0, LSE = -inf.  A q_lens entry
+ *            outside [0, q_len] is clamped and sets MLA_ERR_INVALID_ARG in the
+ *            status word.
+ * All other arguments, layouts and errors as for mla_decode_fwd (which is this
+ * call with q_lens = NULL); q_lens must be 4-byte aligned.
+ */
+MLA_API int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *seqlens, const int32_t *q_lens,
+                          const int32_t *block_table, int batch, int q_len, int num_heads, int64_t kv_rows,
+                          int max_blocks, float softmax_scale, int causal, void *o, float *lse,
+                          void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream);
+
+/*
  * Log-sum-exp merge of the split-KV partials that mla_decode_fwd left in the
  * workspace: lse = ln sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s, for
  * every sequence split over several CTAs; also writes O = 0, LSE = -inf for

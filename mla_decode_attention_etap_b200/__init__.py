@@ -28,7 +28,7 @@ STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3:
 
 EXPORTS = ("mla_decode_workspace_size", "mla_decode_plan", "mla_decode_fwd", "mla_combine",
            "mla_decode_read_status", "mla_decode_plan_host", "mla_status_string", "mla_last_cuda_error",
-           "mla_decode_fwd_static_ws")
+           "mla_decode_fwd_static_ws", "mla_decode_fwd_ragged")
 STATIC_WORKSPACE_BYTES = 8388608
 
 
@@ -57,6 +57,9 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp, vp, vp, sz,
                                      i32, ctypes.c_uint, vp]
         L.mla_decode_fwd.restype = i32
+        L.mla_decode_fwd_ragged.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp, vp,
+                                            vp, sz, i32, ctypes.c_uint, vp]
+        L.mla_decode_fwd_ragged.restype = i32
         L.mla_combine.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
         L.mla_combine.restype = i32
         L.mla_decode_read_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
@@ -110,16 +113,25 @@ def mla_decode_plan(seqlens: torch.Tensor, q_len: int, num_heads: int, workspace
 
 
 def mla_decode_fwd(q, kv, seqlens, block_table, softmax_scale, causal, o, lse, workspace, n_sms, flags=0,
-                   stream=None) -> None:
+                   stream=None, q_lens=None) -> None:
+    """``q_lens`` (optional int32 device tensor [B]): ragged batch, q_lens[b] real query tokens of the
+    q_len rows of sequence b (``mla_decode_fwd_ragged``)."""
     B, q_len, h, _ = q.shape
     if block_table is not None:
         kv_rows, max_blocks = kv.shape[0] * kv.shape[1], block_table.shape[1]
     else:
         kv_rows, max_blocks = kv.shape[1], 0
-    _check(lib().mla_decode_fwd(_ptr(q), _ptr(kv), _ptr(seqlens), _ptr(block_table), B, q_len, h, kv_rows,
-                                max_blocks, float(softmax_scale), int(bool(causal)), _ptr(o), _ptr(lse),
-                                _ptr(workspace), workspace.numel() * workspace.element_size(), n_sms, flags,
-                                _stream(stream)), "mla_decode_fwd")
+    if q_lens is None:
+        _check(lib().mla_decode_fwd(_ptr(q), _ptr(kv), _ptr(seqlens), _ptr(block_table), B, q_len, h, kv_rows,
+                                    max_blocks, float(softmax_scale), int(bool(causal)), _ptr(o), _ptr(lse),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), n_sms, flags,
+                                    _stream(stream)), "mla_decode_fwd")
+    else:
+        _check(lib().mla_decode_fwd_ragged(_ptr(q), _ptr(kv), _ptr(seqlens), _ptr(q_lens), _ptr(block_table), B,
+                                           q_len, h, kv_rows, max_blocks, float(softmax_scale), int(bool(causal)),
+                                           _ptr(o), _ptr(lse), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), n_sms, flags,
+                                           _stream(stream)), "mla_decode_fwd_ragged")
 
 
 def mla_combine(workspace, batch, q_len, num_heads, n_sms, o, lse, stream=None) -> None:
@@ -163,7 +175,7 @@ class MlaDecoder:
         mla_decode_plan(seqlens, self.q_len, self.num_heads, self.workspace, self.n_sms, stream)
 
     def fwd(self, q, kv, seqlens, block_table=None, softmax_scale=None, causal=False, o=None, lse=None,
-            flags=0, stream=None):
+            flags=0, stream=None, q_lens=None):
         B, q_len, h, _ = q.shape
         if o is None:
             o = torch.empty(B, q_len, h, D_V, dtype=torch.bfloat16, device=q.device)
@@ -171,15 +183,15 @@ class MlaDecoder:
             lse = torch.empty(B, q_len, h, dtype=torch.float32, device=q.device)
         scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(D_QK)
         mla_decode_fwd(q, kv, seqlens, block_table, scale, causal, o, lse, self.workspace, self.n_sms, flags,
-                       stream)
+                       stream, q_lens=q_lens)
         return o, lse
 
     def status(self, stream=None) -> int:
         return mla_decode_read_status(self.workspace, stream)
 
 
-def mla_decode(q, kv, seqlens, block_table=None, softmax_scale=None, causal=False):
+def mla_decode(q, kv, seqlens, block_table=None, softmax_scale=None, causal=False, q_lens=None):
     """One-shot convenience: plan + decode (+ combine).  Returns (O bf16, LSE fp32)."""
     dec = MlaDecoder(q.shape[0], q.shape[1], q.shape[2], device=q.device)
     dec.plan(seqlens)
-    return dec.fwd(q, kv, seqlens, block_table, softmax_scale, causal)
+    return dec.fwd(q, kv, seqlens, block_table, softmax_scale, causal, q_lens=q_lens)

@@ -35,6 +35,7 @@ struct WaitCtl {
 
 struct DecodeParams {
     const int32_t *seqlens;
+    const int32_t *q_lens;  // ragged batch: query tokens per sequence (<= q_len), or NULL
     const int32_t *block_table;
     int32_t *ws;  // workspace (int32 view)
     float *opart;

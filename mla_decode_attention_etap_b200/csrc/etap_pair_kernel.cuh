@@ -554,7 +554,29 @@ __global__ void __launch_bounds__(320, 1)
                 int L = p.seqlens[b];
                 if ((int64_t)L > l_cap) L = (int)l_cap;
                 if (L < 0) L = 0;
+                // query tokens of this sequence: all q_len, or q_lens[b] of them (ragged batch; the
+                // rest are padding columns that see no row)
+                int qlen_b = p.q_len;
+                if (p.q_lens) {
+                    qlen_b = p.q_lens[b];
+                    if (qlen_b < 0 || qlen_b > p.q_len) {
+                        if (row == 0 && half == 0) atomicCAS(status, 0, kStatusInvalid);
+                        qlen_b = qlen_b < 0 ? 0 : p.q_len;
+                    }
+                }
                 float m[NH], lpart[NH];  // index 8*ch + n  <->  column 16*ch + 8*half + n
+                // visible rows of this warp's columns (0 for padding and absent columns): lane li holds
+                // that of the warp's li-th column (all lanes of a warp handle the same columns)
+                static_assert(NH <= 32, "one column per lane");
+                int vis_lane = 0;
+                if (lane < NH) {
+                    const int ng = grp * NG + 16 * (lane >> 3) + 8 * half + (lane & 7);
+                    if (ng < p.ncols) {
+                        const int tok = ng / p.num_heads;
+                        vis_lane = tok >= qlen_b ? 0 : (p.causal ? (L - qlen_b + tok + 1) : L);
+                        vis_lane = vis_lane < 0 ? 0 : vis_lane;
+                    }
+                }
 #pragma unroll
                 for (int n = 0; n < NH; ++n) {
                     m[n] = -INFINITY;
@@ -567,7 +589,8 @@ __global__ void __launch_bounds__(320, 1)
                     tc_fence_after();
                     const int rg = t * kTileRows + row;
                     // every row of the tile visible to every column: no per-column mask needed
-                    const bool full_tile = (t + 1) * kTileRows <= (p.causal ? L - p.q_len + 1 : L);
+                    const bool full_tile =
+                        qlen_b == p.q_len && (t + 1) * kTileRows <= (p.causal ? L - qlen_b + 1 : L);
                     bool waited_prev = false, rescale_any = false, sent_next = false;
                     float xc[C::CH][8];  // CH > 1: full scores of this thread's columns, in registers
                     if constexpr (C::CH > 1) {
@@ -645,12 +668,7 @@ __global__ void __launch_bounds__(320, 1)
                         } else {
 #pragma unroll
                             for (int n = 0; n < 8; ++n) {
-                                const int ng = grp * NG + 16 * ch + 8 * half + n;
-                                int vis = 0;
-                                if (ng < p.ncols) {
-                                    vis = p.causal ? (L - p.q_len + ng / p.num_heads + 1) : L;
-                                    vis = vis < 0 ? 0 : vis;
-                                }
+                                const int vis = __shfl_sync(0xffffffffu, vis_lane, 8 * ch + n);
                                 x[n] = (rg < vis) ? x[n] * p.scale_log2 : -INFINITY;
                             }
                         }

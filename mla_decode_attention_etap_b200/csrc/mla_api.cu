@@ -233,6 +233,14 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
                    int q_len, int num_heads, int64_t kv_rows, int max_blocks, float softmax_scale, int causal,
                    void *o, float *lse, void *workspace, size_t workspace_bytes, int num_sms, unsigned flags,
                    void *stream) {
+    return mla_decode_fwd_ragged(q, kv, seqlens, nullptr, block_table, batch, q_len, num_heads, kv_rows, max_blocks,
+                                 softmax_scale, causal, o, lse, workspace, workspace_bytes, num_sms, flags, stream);
+}
+
+int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *seqlens, const int32_t *q_lens,
+                          const int32_t *block_table, int batch, int q_len, int num_heads, int64_t kv_rows,
+                          int max_blocks, float softmax_scale, int causal, void *o, float *lse, void *workspace,
+                          size_t workspace_bytes, int num_sms, unsigned flags, void *stream) {
     int st = check_shape(batch, q_len, num_heads, num_sms);
     if (st != MLA_OK) return st;
     if (!q || !kv || !seqlens || !o || !lse || !workspace) return MLA_ERR_INVALID_ARG;
@@ -249,7 +257,7 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
         if ((int64_t)batch * kv_rows > INT32_MAX) return MLA_ERR_UNSUPPORTED;
     }
     if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(o, 16) || !aligned(lse, 4) || !aligned(seqlens, 4) ||
-        !aligned(workspace, 256))
+        !aligned(workspace, 256) || !aligned(q_lens, 4))
         return MLA_ERR_ALIGNMENT;
     const mla::WsLayout lay = mla::ws_layout(batch, q_len, num_heads, num_sms);
     if (workspace_bytes < lay.total) return MLA_ERR_WORKSPACE;
@@ -272,6 +280,7 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
     char *ws = reinterpret_cast<char *>(workspace);
     mla::DecodeParams p{};
     p.seqlens = seqlens;
+    p.q_lens = q_lens;
     p.block_table = block_table;
     p.ws = reinterpret_cast<int32_t *>(ws);
     p.opart = reinterpret_cast<float *>(ws + lay.opart);

@@ -46,6 +46,7 @@ class Workload:
     num_heads: int
     causal: bool
     softmax_scale: float
+    q_lens: Optional[torch.Tensor] = None  # ragged batch: real query tokens per sequence (int32 [B])
 
     @property
     def batch(self) -> int:
@@ -99,6 +100,7 @@ def make_workload(
     l_max: Optional[int] = None,
     softmax_scale: Optional[float] = None,
     extra_blocks: int = 0,
+    q_lens: Optional[Sequence[int]] = None,
 ) -> Workload:
     """Draw one synthetic MLA decode batch.
 
@@ -140,8 +142,12 @@ def make_workload(
                 off_in = (rows % PAGE).to(kv.device)
                 kv[blk, off_in] = (kv[blk, off_in].float() * spike_scale).to(torch.bfloat16)
     scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(D_QK)
+    ql = None
+    if q_lens is not None:
+        assert len(q_lens) == batch and all(0 <= int(x) <= q_len for x in q_lens)
+        ql = torch.tensor([int(x) for x in q_lens], dtype=torch.int32)
     return Workload(q=q, kv=kv, seqlens=seqlens_t, block_table=block_table, q_len=q_len,
-                    num_heads=num_heads, causal=causal, softmax_scale=scale)
+                    num_heads=num_heads, causal=causal, softmax_scale=scale, q_lens=ql)
 
 
 # The five synthetic workloads (sizes follow the DeepSeek-R1 MLA decode shape).
@@ -173,6 +179,15 @@ def workload_b16_h16_q4_causal(seed: int = 0, device="cpu", seqlen: int = 32768,
                          spike_frac=0.05, spike_scale=8.0)
 
 
+def workload_b16_h16_ragged_q4_causal(seed: int = 0, device="cpu", seqlen: int = 32768,
+                                      batch: int = 16) -> Workload:
+    """Ragged speculative verify: B=16, 16 heads, 1..4 causal query tokens per sequence (uniform,
+    from ``seed + 3``) at the end of a 32768-row cache, 5% of rows scaled x8."""
+    q_lens = draw_seqlens(batch, 1, 4, seed + 3)
+    return make_workload(batch, 16, [seqlen] * batch, q_len=4, causal=True, seed=seed, device=device,
+                         spike_frac=0.05, spike_scale=8.0, q_lens=q_lens)
+
+
 def bf16_bits(t: torch.Tensor):
     """uint16 numpy view of a bf16 tensor (CPU), for the oracle's C interface."""
     import numpy as np
@@ -184,12 +199,15 @@ def algorithmic_kv_bytes(seqlens: Sequence[int]) -> int:
     return sum(int(L) for L in seqlens) * D_QK * 2
 
 
-def algorithmic_flops(seqlens: Sequence[int], q_len: int, num_heads: int, causal: bool) -> int:
-    """2*(576+512) flops per visible (query column, KV token) pair."""
+def algorithmic_flops(seqlens: Sequence[int], q_len: int, num_heads: int, causal: bool,
+                      q_lens: Optional[Sequence[int]] = None) -> int:
+    """2*(576+512) flops per visible (query column, KV token) pair (padding tokens of a ragged
+    batch see no pair)."""
     total = 0
-    for L in seqlens:
+    for b, L in enumerate(seqlens):
         L = int(L)
-        for t in range(q_len):
-            vis = (L - q_len + t + 1) if causal else L
+        qb = q_len if q_lens is None else int(q_lens[b])
+        for t in range(qb):
+            vis = (L - qb + t + 1) if causal else L
             total += max(vis, 0) * num_heads
     return total * 2 * (D_QK + D_V)

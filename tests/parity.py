@@ -30,7 +30,8 @@ def run_cuda(w: Workload, n_sms=None, flags=0, poison=True, decoder=None):
     lse = torch.full((w.batch, w.q_len, w.num_heads), float("nan") if poison else 0.0,
                      dtype=torch.float32, device=dev)
     dec.plan(sl)
-    dec.fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o=o, lse=lse, flags=flags)
+    ql = w.q_lens.to(dev) if w.q_lens is not None else None
+    dec.fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o=o, lse=lse, flags=flags, q_lens=ql)
     torch.cuda.synchronize()
     status = dec.status()
     return o.float().cpu().numpy(), lse.cpu().numpy(), status, dec
@@ -42,14 +43,16 @@ def run_oracle(w: Workload, batch_index=None):
         q = bf16_bits(w.q)
         kv = bf16_bits(w.kv)
         bt = None if w.block_table is None else w.block_table.numpy()
-        return om.mla_decode(q, kv, w.seqlens.numpy(), bt, w.softmax_scale, w.causal)
+        ql = None if w.q_lens is None else w.q_lens.numpy()
+        return om.mla_decode(q, kv, w.seqlens.numpy(), bt, w.softmax_scale, w.causal, q_lens=ql)
     outs_o, outs_l = [], []
     for b in batch_index:
         L = int(w.seqlens[b])
         rows = w.kv_rows(b).cpu()
         kv = bf16_bits(rows.reshape(1, max(L, 0), 576)) if L > 0 else np.zeros((1, 1, 576), np.uint16)
         q = bf16_bits(w.q[b:b + 1].cpu())
-        o, lse = om.mla_decode(q, kv, np.array([L], np.int32), None, w.softmax_scale, w.causal)
+        ql = None if w.q_lens is None else w.q_lens[b:b + 1].numpy()
+        o, lse = om.mla_decode(q, kv, np.array([L], np.int32), None, w.softmax_scale, w.causal, q_lens=ql)
         outs_o.append(o[0])
         outs_l.append(lse[0])
     return np.stack(outs_o), np.stack(outs_l)

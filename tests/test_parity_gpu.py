@@ -280,3 +280,31 @@ def test_many_column_groups(heads, q_len, causal):
     o, lse, st, _ = run_cuda(w)
     assert st == 0
     assert_parity(o, lse, *run_oracle(w), what=f"h={heads} q={q_len}")
+
+
+@pytest.mark.parametrize("heads,q_len,causal,paged", [(16, 1, False, False), (4, 4, True, False), (4, 4, False, True),
+                                                      (16, 4, True, False), (16, 4, True, True), (32, 3, True, False)])
+def test_ragged_q_lens(heads, q_len, causal, paged):
+    """Ragged multi-token decode: per-sequence token counts 0..q_len (16- and 32-column groups)."""
+    lens = [900, 3, 130, 257, 64]
+    q_lens = [q_len, 0, 1, max(q_len - 1, 0), q_len]
+    w = _poison_padding(W.make_workload(len(lens), heads, lens, q_len=q_len, causal=causal, paged=paged,
+                                        seed=40 + heads + q_len, q_lens=q_lens, spike_frac=0.05))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    o_ref, lse_ref = run_oracle(w)
+    for b, qb in enumerate(q_lens):          # padding tokens: exact zeros and -inf
+        assert np.all(o[b, qb:] == 0) and np.all(np.isneginf(lse[b, qb:]))
+    assert_parity(o, lse, o_ref, lse_ref, what=f"ragged h={heads} q={q_len}")
+
+
+def test_ragged_q_lens_out_of_range_sets_status():
+    w = W.make_workload(2, 16, [300, 200], q_len=2, seed=50, q_lens=[2, 1])
+    w.q_lens[1] = 7                          # more tokens than q_len
+    _, _, st, _ = run_cuda(w)
+    assert st == -1                          # MLA_ERR_INVALID_ARG in the status word
+
+
+def test_full_b16_h16_ragged_q4_causal_sampled():
+    w = W.workload_b16_h16_ragged_q4_causal(seed=0, device="cuda")
+    _full(w, [0, 5, 13])
