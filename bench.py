@@ -361,6 +361,24 @@ def run_ours(args):
         for i in range(args.steps):
             step(i)
         torch.cuda.synchronize()
+        # attainable read bandwidth of the decode's TMA pattern on this GPU: the streaming probe
+        # (same grid, split, slots and L2 prefetch, no computation) over the same cache tensor
+        kv_flat = kv.reshape(-1, 576)
+        probe_rows = (kv_flat.shape[0] // 128) * 128
+        probe_err = torch.zeros(1, dtype=torch.int32, device=dev)
+        probe_units = dec.n_sms // 2
+        for _ in range(3):
+            mla.mla_stream_probe(kv_flat[:probe_rows], probe_units, probe_err)
+        pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pe0.record(stream)
+        n_probe = max(3, min(args.steps, 50))
+        for _ in range(n_probe):
+            mla.mla_stream_probe(kv_flat[:probe_rows], probe_units, probe_err)
+        pe1.record(stream)
+        torch.cuda.synchronize()
+        probe_s = pe0.elapsed_time(pe1) / 1e3 / n_probe
+        if int(probe_err.item()) != 0:
+            raise RuntimeError("streaming probe: a bounded wait ran out")
     status = dec.status()
     if status != 0:
         raise RuntimeError(f"device status {mla.STATUS.get(status, status)}")
@@ -422,6 +440,10 @@ def run_ours(args):
             roof = {"bound": "tensor", "achieved": ach, "peak": tc_tflops, "unit": "TFLOP/s", "frac": ach / tc_tflops}
         roof["traffic"] = profiled_traffic(wname)
         roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+        roof["attainable_read_gbs"] = probe_rows * 1152 / probe_s / 1e9
+        roof["frac_of_attainable"] = roof["achieved"] / roof["attainable_read_gbs"] if bound == "hbm" else None
+        roof["attainable_note"] = ("streaming probe: the decode's TMA read pattern (same grid, column split, "
+                                   "5 V-pair slots, L2 prefetch) without computation, over the same cache")
         roof["kernel"] = "etap_pair_kernel"
         roof["kernel_ms"] = kern_s * 1e3
         roof["kernel_timing"] = ("CUDA events on the launch stream around each of K decode launches, "

@@ -159,6 +159,17 @@ MLA_API int mla_combine(const void *workspace, int batch, int q_len, int num_hea
                 void *o, float *lse, void *stream);
 
 /*
+ * Measurement helper, not part of the decode (the pages have no counterpart): streams
+ * rows x 576 bf16 (kv, 16-byte aligned, rows a multiple of 128, < 2^31) with exactly
+ * the decode kernel's TMA read pattern (2*units CTAs, each CTA pair splitting every
+ * 128-row tile by latent columns, 5 V-pair slots, L2 prefetch one tile ahead) and no
+ * computation, so that timing it gives the read bandwidth that pattern can reach.
+ * err: device int32, zeroed by the caller, set to 1 if a bounded wait ran out.
+ * Asynchronous on `stream`; allocates nothing.
+ */
+MLA_API int mla_stream_probe(const void *kv, int64_t rows, int units, int32_t *err, void *stream);
+
+/*
  * Copy the workspace status word to the host (waits for that copy only).
  * *status_out receives MLA_OK or the first device-side error recorded.
  */

@@ -28,7 +28,7 @@ STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3:
 
 EXPORTS = ("mla_decode_workspace_size", "mla_decode_plan", "mla_decode_fwd", "mla_combine",
            "mla_decode_read_status", "mla_decode_plan_host", "mla_status_string", "mla_last_cuda_error",
-           "mla_decode_fwd_static_ws", "mla_decode_fwd_ragged")
+           "mla_decode_fwd_static_ws", "mla_decode_fwd_ragged", "mla_stream_probe")
 STATIC_WORKSPACE_BYTES = 8388608
 
 
@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_fwd_static_ws.argtypes = [vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp,
                                                vp, i32, vp]
         L.mla_decode_fwd_static_ws.restype = i32
+        L.mla_stream_probe.argtypes = [vp, i64, i32, vp, vp]
+        L.mla_stream_probe.restype = i32
         L.mla_last_cuda_error.argtypes = []
         L.mla_last_cuda_error.restype = ctypes.c_char_p
         _lib = L
@@ -132,6 +134,13 @@ def mla_decode_fwd(q, kv, seqlens, block_table, softmax_scale, causal, o, lse, w
                                            _ptr(o), _ptr(lse), _ptr(workspace),
                                            workspace.numel() * workspace.element_size(), n_sms, flags,
                                            _stream(stream)), "mla_decode_fwd_ragged")
+
+
+def mla_stream_probe(kv, units: int, err, stream=None) -> None:
+    """Stream ``kv`` ([..., 576] bf16, rows a multiple of 128) with the decode's TMA read pattern and
+    no computation (a bandwidth probe).  ``err``: int32 device tensor [1], zeroed by the caller."""
+    rows = kv.numel() // 576
+    _check(lib().mla_stream_probe(_ptr(kv), rows, units, _ptr(err), _stream(stream)), "mla_stream_probe")
 
 
 def mla_combine(workspace, batch, q_len, num_heads, n_sms, o, lse, stream=None) -> None:

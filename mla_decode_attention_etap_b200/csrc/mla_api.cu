@@ -16,6 +16,7 @@
 #include "etap_pair_kernel.cuh"
 #include "plan_combine_kernels.cuh"
 #include "plan_core.h"
+#include "stream_probe.cuh"
 
 namespace {
 
@@ -317,6 +318,30 @@ int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *seqlens,
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
     if (separate_combine) return mla_combine(workspace, batch, q_len, num_heads, num_sms, o, lse, stream);
+    return MLA_OK;
+}
+
+int mla_stream_probe(const void *kv, int64_t rows, int units, int32_t *err, void *stream) {
+    if (!kv || !err) return MLA_ERR_INVALID_ARG;
+    if (rows < 128 || rows % 128 != 0 || rows > INT32_MAX || units < 1 || units > 4096) return MLA_ERR_INVALID_ARG;
+    if (!aligned(kv, 16) || !aligned(err, 4)) return MLA_ERR_ALIGNMENT;
+    CUtensorMap tm_kv, tm_kvr;
+    int st = encode_rows_576(&tm_kv, kv, (uint64_t)rows, 64);
+    if (st != MLA_OK) return st;
+    st = encode_rows_576(&tm_kvr, kv, (uint64_t)rows, 64, 32);
+    if (st != MLA_OK) return st;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(mla::stream_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)mla::kProbeSmem);
+    });
+    if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute");
+    mla::ProbeParams pp{rows, units, err};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    mla::stream_probe_kernel<<<2 * units, 64, mla::kProbeSmem, s>>>(tm_kv, tm_kvr, pp);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "stream_probe_kernel launch");
     return MLA_OK;
 }
 

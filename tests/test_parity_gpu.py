@@ -308,3 +308,14 @@ def test_ragged_q_lens_out_of_range_sets_status():
 def test_full_b16_h16_ragged_q4_causal_sampled():
     w = W.workload_b16_h16_ragged_q4_causal(seed=0, device="cuda")
     _full(w, [0, 5, 13])
+
+
+def test_stream_probe_runs_clean():
+    """The bandwidth probe (decode's TMA pattern without computation) completes with no expired wait."""
+    import mla_decode_attention_etap_b200 as mla
+    kv = torch.zeros(16 * 4096, 576, dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for units in (74, 3):
+        mla.mla_stream_probe(kv, units, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
