@@ -554,6 +554,9 @@ __global__ void __launch_bounds__(320, 1)
                 int L = p.seqlens[b];
                 if ((int64_t)L > l_cap) L = (int)l_cap;
                 if (L < 0) L = 0;
+                // split bookkeeping of this sequence, read now so that the epilogue does not wait for it
+                const int seg_nsplit = seq_info[4 * b + 2];
+                const int seg_slot = seq_info[4 * b + 3] + (unit - seq_info[4 * b + 1]);
                 // query tokens of this sequence: all q_len, or q_lens[b] of them (ragged batch; the
                 // rest are padding columns that see no row)
                 int qlen_b = p.q_len;
@@ -822,8 +825,8 @@ __global__ void __launch_bounds__(320, 1)
                     stop = true;
                     break;
                 }
-                const int nsplit = seq_info[4 * b + 2];
-                const int slot = seq_info[4 * b + 3] + (unit - seq_info[4 * b + 1]);
+                const int nsplit = seg_nsplit;
+                const int slot = seg_slot;
 #pragma unroll
                 for (int ch = 0; ch < C::CH; ++ch) {
                     float inv_l[8], lse_n[8];
