@@ -319,3 +319,35 @@ def test_stream_probe_runs_clean():
         mla.mla_stream_probe(kv, units, err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
+
+
+def test_cuda_graph_replay_matches_eager():
+    """plan + fwd captured once in a CUDA graph (programmatic launches become graph edges) and
+    replayed: bitwise the eager result, repeatedly (the merge counters reset themselves)."""
+    from mla_decode_attention_etap_b200 import MlaDecoder
+    w = W.make_workload(3, 16, [5000, 700, 2100], seed=60)
+    dev = torch.device("cuda")
+    q, kv, sl = w.q.to(dev), w.kv.to(dev), w.seqlens.to(dev)
+    dec = MlaDecoder(w.batch, w.q_len, w.num_heads, device=dev)
+    o = torch.empty(w.batch, 1, 16, 512, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(w.batch, 1, 16, dtype=torch.float32, device=dev)
+    dec.plan(sl)
+    dec.fwd(q, kv, sl, None, w.softmax_scale, False, o=o, lse=lse)
+    torch.cuda.synchronize()
+    o_eager, l_eager = o.clone(), lse.clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        o.zero_()
+        with torch.cuda.graph(g, stream=side):
+            dec.plan(sl, stream=side)
+            dec.fwd(q, kv, sl, None, w.softmax_scale, False, o=o, lse=lse, stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(3):
+        o.zero_()
+        lse.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_eager) and torch.equal(lse, l_eager)
+    assert dec.status() == 0
