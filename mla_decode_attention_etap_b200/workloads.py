@@ -21,6 +21,12 @@ Recipe (one ``torch.Generator`` seeded with ``seed``, drawn in this order):
   5. the "spike" rows: a fraction of each sequence's KV rows (chosen by a
      per-sequence permutation) multiplied by ``spike_scale`` (exact in bf16 for
      powers of two).
+
+FP8 caches (``kv_dtype="e4m3"``) quantise that bf16 cache row by row (no further
+random draws): scale[r] = max_k |kv[r, k]| / 448 in fp32 (1 for an all-zero row)
+and code[r, k] = E4M3(kv[r, k] / scale[r]) rounded to nearest-even, so every
+row uses the full E4M3 range.  ``kv8`` holds the codes (uint8, same layout as
+``kv``) and ``kv_scale`` the fp32 scales ([B, L_max] or [num_blocks, 64]).
 """
 
 from __future__ import annotations
@@ -47,6 +53,12 @@ class Workload:
     causal: bool
     softmax_scale: float
     q_lens: Optional[torch.Tensor] = None  # ragged batch: real query tokens per sequence (int32 [B])
+    kv8: Optional[torch.Tensor] = None      # FP8 cache: E4M3 codes, uint8, laid out like kv
+    kv_scale: Optional[torch.Tensor] = None  # FP8 cache: fp32 scale per cache row
+
+    @property
+    def fp8(self) -> bool:
+        return self.kv8 is not None
 
     @property
     def batch(self) -> int:
@@ -101,6 +113,7 @@ def make_workload(
     softmax_scale: Optional[float] = None,
     extra_blocks: int = 0,
     q_lens: Optional[Sequence[int]] = None,
+    kv_dtype: str = "bf16",
 ) -> Workload:
     """Draw one synthetic MLA decode batch.
 
@@ -146,8 +159,27 @@ def make_workload(
     if q_lens is not None:
         assert len(q_lens) == batch and all(0 <= int(x) <= q_len for x in q_lens)
         ql = torch.tensor([int(x) for x in q_lens], dtype=torch.int32)
+    kv8 = kv_scale = None
+    if kv_dtype == "e4m3":
+        kv8, kv_scale = quantize_e4m3_rows(kv)
+    else:
+        assert kv_dtype == "bf16", kv_dtype
     return Workload(q=q, kv=kv, seqlens=seqlens_t, block_table=block_table, q_len=q_len,
-                    num_heads=num_heads, causal=causal, softmax_scale=scale, q_lens=ql)
+                    num_heads=num_heads, causal=causal, softmax_scale=scale, q_lens=ql, kv8=kv8,
+                    kv_scale=kv_scale)
+
+
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3_rows(kv: torch.Tensor):
+    """Per-row E4M3 quantisation of a [..., 576] cache -> (codes uint8 [..., 576], scale fp32 [...])."""
+    x = kv.float()
+    amax = x.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    y = (x / scale[..., None]).clamp(-E4M3_MAX, E4M3_MAX)
+    codes = y.to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale.contiguous()
 
 
 # The five synthetic workloads (sizes follow the DeepSeek-R1 MLA decode shape).
@@ -188,15 +220,28 @@ def workload_b16_h16_ragged_q4_causal(seed: int = 0, device="cpu", seqlen: int =
                          spike_frac=0.05, spike_scale=8.0, q_lens=q_lens)
 
 
+def workload_b16_h16_fp8(seqlen: int, seed: int = 0, device="cpu") -> Workload:
+    """B=16, 16 heads, one query token, equal contiguous lengths, FP8 (E4M3 + row scale) cache."""
+    return make_workload(16, 16, [seqlen] * 16, seed=seed, device=device, kv_dtype="e4m3")
+
+
+def workload_b64_h16_paged_fp8(seed: int = 0, device="cpu", batch: int = 64, lmax: int = 65536) -> Workload:
+    """The B=64 paged workload with an FP8 (E4M3 + row scale) cache."""
+    lens = draw_seqlens(batch, 1, lmax, seed)
+    return make_workload(batch, 16, lens, paged=True, seed=seed, device=device, kv_dtype="e4m3")
+
+
 def bf16_bits(t: torch.Tensor):
     """uint16 numpy view of a bf16 tensor (CPU), for the oracle's C interface."""
     import numpy as np
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def algorithmic_kv_bytes(seqlens: Sequence[int]) -> int:
-    """KV bytes a decode step must read once: 576 bf16 values per cached token."""
-    return sum(int(L) for L in seqlens) * D_QK * 2
+def algorithmic_kv_bytes(seqlens: Sequence[int], fp8: bool = False) -> int:
+    """KV bytes a decode step must read once: 576 bf16 values per cached token, or 576 E4M3
+    codes and one fp32 scale."""
+    per_token = D_QK + 4 if fp8 else D_QK * 2
+    return sum(int(L) for L in seqlens) * per_token
 
 
 def algorithmic_flops(seqlens: Sequence[int], q_len: int, num_heads: int, causal: bool,

@@ -30,6 +30,13 @@
  * Inputs are bf16 bit patterns (uint16), widened exactly to fp64.  All
  * arithmetic is fp64.  Paged caches ([num_blocks, page, 576]) are resolved
  * through the block table; contiguous caches are [B, kv_rows, 576].
+ *
+ * FP8 latent cache (an adjacent storage format; the pages keep the cache in
+ * bf16): every cache row is 576 OCP FP8 E4M3 codes plus one fp32 scale for the
+ * row, and element k of row r stands for scale[r] * e4m3(code[r][k]).  The
+ * oracle widens every element to that fp64 value and then computes exactly the
+ * definition above; the scale array is indexed like the rows ([B, kv_rows], or
+ * [num_blocks, page] when paged).
  */
 #include <math.h>
 #include <stdint.h>
@@ -55,6 +62,49 @@ static const uint16_t *kv_row(const uint16_t *kv, const int32_t *block_table, in
     return kv + ((int64_t)b * kv_rows + j) * d_qk;
 }
 
+/*
+ * OCP 8-bit floating point, E4M3 variant: 1 sign bit, 4 exponent bits (bias 7),
+ * 3 mantissa bits, no infinities; exponent 0 is subnormal (m/8 * 2^-6) and the
+ * all-ones exponent and mantissa (0x7F, 0xFF) is NaN.  Largest finite value 448.
+ */
+static double e4m3_to_double(uint8_t code)
+{
+    int e = (code >> 3) & 0xF, m = code & 7;
+    double v;
+    if (e == 0xF && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);          /* (m / 8) * 2^-6 */
+    else
+        v = ldexp((double)(8 + m), e - 10); /* (1 + m / 8) * 2^(e - 7) */
+    return (code & 0x80) ? -v : v;
+}
+
+/* A latent cache in either storage format. */
+typedef struct {
+    const uint16_t *bf16;     /* bf16 bit patterns, or NULL */
+    const uint8_t *e4m3;      /* E4M3 codes (with row_scale), or NULL */
+    const float *row_scale;   /* one scale per cache row */
+    const double *e4m3_value; /* [256] decoded codes */
+    const int32_t *block_table;
+    int kv_rows, max_blocks, page, d_qk;
+} kv_cache;
+
+/* Widen the first n values of row j of sequence b to fp64. */
+static void widen_row(const kv_cache *c, int b, int j, int n, double *dst)
+{
+    int64_t r = c->block_table
+                    ? (int64_t)c->block_table[(int64_t)b * c->max_blocks + j / c->page] * c->page + j % c->page
+                    : (int64_t)b * c->kv_rows + j;
+    if (c->e4m3) {
+        const uint8_t *src = c->e4m3 + r * c->d_qk;
+        double s = (double)c->row_scale[r];
+        for (int k = 0; k < n; ++k) dst[k] = s * c->e4m3_value[src[k]];
+    } else {
+        const uint16_t *src = c->bf16 + r * c->d_qk;
+        for (int k = 0; k < n; ++k) dst[k] = bf16_to_double(src[k]);
+    }
+}
+
 static int visible_rows(int L, int q_len, int t, int causal)
 {
     int vis = causal ? (L - q_len + t + 1) : L;
@@ -70,10 +120,16 @@ static int token_visible_rows(int L, int q_len, const int32_t *q_lens, int b, in
     return visible_rows(L, qb, t, causal);
 }
 
-static int decode_standard(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
-                           const int32_t *q_lens, const int32_t *block_table, int B, int q_len, int h,
-                           int d_qk, int d_v, int kv_rows, int max_blocks, int page, double scale,
+static int decode_standard(const uint16_t *q, const kv_cache *c, const int32_t *seqlens,
+                           const int32_t *q_lens, int B, int q_len, int h, int d_v, double scale,
                            int causal, double *o, double *lse);
+
+static kv_cache bf16_cache(const uint16_t *kv, const int32_t *block_table, int kv_rows, int max_blocks,
+                           int page, int d_qk)
+{
+    kv_cache c = {kv, NULL, NULL, NULL, block_table, kv_rows, max_blocks, page, d_qk};
+    return c;
+}
 
 /*
  * Standard form: S = Q K^T, P = softmax(S) over the KV axis, O = P V.
@@ -85,8 +141,8 @@ int oracle_mla_decode(const uint16_t *q, const uint16_t *kv, const int32_t *seql
                       int kv_rows, int max_blocks, int page, double scale, int causal,
                       double *o, double *lse)
 {
-    return decode_standard(q, kv, seqlens, NULL, block_table, B, q_len, h, d_qk, d_v, kv_rows,
-                           max_blocks, page, scale, causal, o, lse);
+    kv_cache c = bf16_cache(kv, block_table, kv_rows, max_blocks, page, d_qk);
+    return decode_standard(q, &c, seqlens, NULL, B, q_len, h, d_v, scale, causal, o, lse);
 }
 
 /* The same with q_lens[b] real query tokens in sequence b (0 <= q_lens[b] <= q_len). */
@@ -95,15 +151,31 @@ int oracle_mla_decode_ragged(const uint16_t *q, const uint16_t *kv, const int32_
                              int h, int d_qk, int d_v, int kv_rows, int max_blocks, int page,
                              double scale, int causal, double *o, double *lse)
 {
-    return decode_standard(q, kv, seqlens, q_lens, block_table, B, q_len, h, d_qk, d_v, kv_rows,
-                           max_blocks, page, scale, causal, o, lse);
+    kv_cache c = bf16_cache(kv, block_table, kv_rows, max_blocks, page, d_qk);
+    return decode_standard(q, &c, seqlens, q_lens, B, q_len, h, d_v, scale, causal, o, lse);
 }
 
-static int decode_standard(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
-                           const int32_t *q_lens, const int32_t *block_table, int B, int q_len, int h,
-                           int d_qk, int d_v, int kv_rows, int max_blocks, int page, double scale,
+/*
+ * FP8 cache: kv8 holds E4M3 codes laid out like the bf16 cache, kv_scale one
+ * fp32 scale per cache row.  q_lens may be NULL (every sequence has q_len
+ * query tokens).
+ */
+int oracle_mla_decode_fp8(const uint16_t *q, const uint8_t *kv8, const float *kv_scale,
+                          const int32_t *seqlens, const int32_t *q_lens, const int32_t *block_table,
+                          int B, int q_len, int h, int d_qk, int d_v, int kv_rows, int max_blocks,
+                          int page, double scale, int causal, double *o, double *lse)
+{
+    double table[256];
+    for (int i = 0; i < 256; ++i) table[i] = e4m3_to_double((uint8_t)i);
+    kv_cache c = {NULL, kv8, kv_scale, table, block_table, kv_rows, max_blocks, page, d_qk};
+    return decode_standard(q, &c, seqlens, q_lens, B, q_len, h, d_v, scale, causal, o, lse);
+}
+
+static int decode_standard(const uint16_t *q, const kv_cache *c, const int32_t *seqlens,
+                           const int32_t *q_lens, int B, int q_len, int h, int d_v, double scale,
                            int causal, double *o, double *lse)
 {
+    int d_qk = c->d_qk;
     int rows = B * q_len * h;
     int failed = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : failed)
@@ -114,7 +186,7 @@ static int decode_standard(const uint16_t *q, const uint16_t *kv, const int32_t 
         int vis = token_visible_rows(L, q_len, q_lens, b, t, causal);
         const uint16_t *qr = q + (int64_t)r * d_qk;
         double *orow = o + (int64_t)r * d_v;
-        double qd[1024];
+        double qd[1024], kd[1024];
         for (int k = 0; k < d_qk; ++k) qd[k] = bf16_to_double(qr[k]);
         for (int d = 0; d < d_v; ++d) orow[d] = 0.0;
         if (vis == 0) {
@@ -128,9 +200,9 @@ static int decode_standard(const uint16_t *q, const uint16_t *kv, const int32_t 
         }
         /* S row: s_j = scale * q . k_j */
         for (int j = 0; j < vis; ++j) {
-            const uint16_t *kr = kv_row(kv, block_table, b, j, kv_rows, max_blocks, page, d_qk);
+            widen_row(c, b, j, d_qk, kd);
             double acc = 0.0;
-            for (int k = 0; k < d_qk; ++k) acc += qd[k] * bf16_to_double(kr[k]);
+            for (int k = 0; k < d_qk; ++k) acc += qd[k] * kd[k];
             s[j] = scale * acc;
         }
         /* softmax over the KV axis, two passes */
@@ -144,9 +216,9 @@ static int decode_standard(const uint16_t *q, const uint16_t *kv, const int32_t 
         }
         /* O = P V with V = the first d_v columns of the latent row */
         for (int j = 0; j < vis; ++j) {
-            const uint16_t *vr = kv_row(kv, block_table, b, j, kv_rows, max_blocks, page, d_qk);
+            widen_row(c, b, j, d_v, kd);
             double p = s[j] / den;
-            for (int d = 0; d < d_v; ++d) orow[d] += p * bf16_to_double(vr[d]);
+            for (int d = 0; d < d_v; ++d) orow[d] += p * kd[d];
         }
         lse[r] = m + log(den);
         free(s);

@@ -14,6 +14,11 @@ Two independent fp64 implementations of the same definition live here:
   to cross-check the C code.
 
 ``lse_merge`` is the log-sum-exp merge of results over disjoint KV ranges.
+
+``mla_decode_fp8`` / ``mla_decode_fp8_numpy`` take an FP8 latent cache (an
+adjacent storage format, not on the pages): E4M3 codes (uint8) plus one fp32
+scale per cache row; element k of row r is scale[r] * e4m3(code[r, k]), and
+the attention is the same definition on those widened values.
 """
 
 from __future__ import annotations
@@ -59,6 +64,9 @@ def _load():
             fn.restype = ctypes.c_int
         lib.oracle_mla_decode_ragged.argtypes = args[:3] + [ctypes.c_void_p] + args[3:]
         lib.oracle_mla_decode_ragged.restype = ctypes.c_int
+        lib.oracle_mla_decode_fp8.argtypes = ([ctypes.c_void_p] * 6 + [ctypes.c_int] * 8 +
+                                              [ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p])
+        lib.oracle_mla_decode_fp8.restype = ctypes.c_int
         lib.oracle_lse_merge.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_lse_merge.restype = None
@@ -113,6 +121,54 @@ def mla_decode_etap(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.0
     return _call("oracle_mla_decode_etap", q_bits, kv_bits, seqlens, block_table, scale, causal)
 
 
+def mla_decode_fp8(q_bits, kv_codes, kv_scale, seqlens, block_table=None, scale=1.0 / 24.0, causal=False,
+                   q_lens=None, threads=None):
+    """Standard-form oracle on an FP8 cache: ``kv_codes`` uint8 E4M3 codes laid out like the bf16
+    cache, ``kv_scale`` fp32 with one scale per cache row ([B, kv_rows] or [num_blocks, 64]).
+    Returns (O fp64 [B,q,h,512], LSE fp64 [B,q,h])."""
+    q_bits = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    kv_codes = np.ascontiguousarray(kv_codes, dtype=np.uint8)
+    kv_scale = np.ascontiguousarray(kv_scale, dtype=np.float32)
+    seqlens = np.ascontiguousarray(seqlens, dtype=np.int32)
+    B, q_len, h, dqk = q_bits.shape
+    assert dqk == D_QK and kv_codes.shape[-1] == D_QK and kv_scale.shape == kv_codes.shape[:-1]
+    if block_table is not None:
+        block_table = np.ascontiguousarray(block_table, dtype=np.int32)
+        kv_rows, max_blocks, page = 0, block_table.shape[1], kv_codes.shape[1]
+    else:
+        kv_rows, max_blocks, page = kv_codes.shape[1], 0, PAGE
+    if q_lens is not None:
+        q_lens = np.ascontiguousarray(q_lens, dtype=np.int32)
+        assert q_lens.shape == (B,) and q_lens.min() >= 0 and q_lens.max() <= q_len
+    o = np.zeros((B, q_len, h, D_V), dtype=np.float64)
+    lse = np.zeros((B, q_len, h), dtype=np.float64)
+    if threads is not None:
+        os.environ["OMP_NUM_THREADS"] = str(threads)
+    rc = _load().oracle_mla_decode_fp8(_ptr(q_bits), _ptr(kv_codes), _ptr(kv_scale), _ptr(seqlens), _ptr(q_lens),
+                                       _ptr(block_table), B, q_len, h, D_QK, D_V, kv_rows, max_blocks, page,
+                                       float(scale), int(bool(causal)), _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise MemoryError(f"oracle_mla_decode_fp8 failed ({rc})")
+    return o, lse
+
+
+def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    """OCP E4M3 codes -> fp64: sign, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0 is
+    subnormal, 0x7F / 0xFF are NaN, there are no infinities."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    e, m = (c >> 3) & 15, c & 7
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return np.where(c & 0x80, -mag, mag)
+
+
+def mla_decode_fp8_numpy(q_bits, kv_codes, kv_scale, seqlens, block_table=None, scale=1.0 / 24.0, causal=False,
+                         q_lens=None):
+    """Second, independent fp64 implementation on the FP8 cache (numpy matmuls on the widened rows)."""
+    kv = e4m3_to_f64(kv_codes) * np.asarray(kv_scale, dtype=np.float64)[..., None]
+    return _decode_numpy_f64(bf16_bits_to_f64(q_bits), kv, seqlens, block_table, scale, causal, q_lens)
+
+
 def lse_merge(o_s: np.ndarray, lse_s: np.ndarray):
     """Merge S partial results over disjoint KV ranges: o_s [S, d], lse_s [S] -> (o [d], lse)."""
     o_s = np.ascontiguousarray(o_s, dtype=np.float64)
@@ -140,8 +196,11 @@ def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
 
 def mla_decode_numpy(q_bits, kv_bits, seqlens, block_table=None, scale=1.0 / 24.0, causal=False, q_lens=None):
     """Second, independent fp64 implementation of the standard form with numpy matmuls."""
-    q = bf16_bits_to_f64(q_bits)
-    kv = bf16_bits_to_f64(kv_bits)
+    return _decode_numpy_f64(bf16_bits_to_f64(q_bits), bf16_bits_to_f64(kv_bits), seqlens, block_table, scale,
+                             causal, q_lens)
+
+
+def _decode_numpy_f64(q, kv, seqlens, block_table, scale, causal, q_lens):
     B, q_len, h, _ = q.shape
     o = np.zeros((B, q_len, h, D_V))
     lse = np.zeros((B, q_len, h))
