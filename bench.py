@@ -58,6 +58,11 @@ WORKLOADS = {
     "b32_h128_paged": dict(kind="b32_h128"),
     "b16_h16_q4_causal": dict(kind="q4_causal"),
     "b16_h16_ragged_q4_causal": dict(kind="ragged_q4_causal"),
+    # FP8 latent cache (E4M3 codes + one fp32 scale per row): 580 bytes per cached token
+    "b16_h16_64k_fp8": dict(batch=16, heads=16, seqlen=65536, fp8=True),
+    "b16_h16_16k_fp8": dict(batch=16, heads=16, seqlen=16384, fp8=True),
+    "b16_h16_4k_fp8": dict(batch=16, heads=16, seqlen=4096, fp8=True),
+    "b64_h16_paged_fp8": dict(kind="b64_paged_fp8"),
 }
 
 
@@ -107,8 +112,14 @@ def make_workload(name: str, rank: int, device):
     if kind == "ragged_q4_causal":
         return (W.workload_b16_h16_ragged_q4_causal(seed=seed, device=device),
                 "mla_decode_b16_h16_ragged_q1to4_causal_L32768_spikes5pct_x8")
-    w = W.make_workload(spec["batch"], spec["heads"], [spec["seqlen"]] * spec["batch"], seed=seed, device=device)
-    return w, f"mla_decode_b{spec['batch']}_h{spec['heads']}_q1_L{spec['seqlen']}_contiguous"
+    if kind == "b64_paged_fp8":
+        return (W.workload_b64_h16_paged_fp8(seed=seed, device=device),
+                "mla_decode_b64_h16_q1_Lunif1to65536_paged64_e4m3cache")
+    fp8 = bool(spec.get("fp8"))
+    w = W.make_workload(spec["batch"], spec["heads"], [spec["seqlen"]] * spec["batch"], seed=seed, device=device,
+                        kv_dtype="e4m3" if fp8 else "bf16")
+    return w, f"mla_decode_b{spec['batch']}_h{spec['heads']}_q1_L{spec['seqlen']}_contiguous" + (
+        "_e4m3cache" if fp8 else "")
 
 
 def load_peaks():
@@ -242,14 +253,13 @@ def oracle_baseline(w, target_s: float = 12.0):
         L = int(w.seqlens[b])
         if L == 0:
             continue
-        rows = w.kv_rows(b).cpu()
-        kv = bf16_bits(rows.reshape(1, L, 576))
         q = bf16_bits(w.q[b:b + 1].cpu())
         ql = None if w.q_lens is None else w.q_lens[b:b + 1].numpy()
+        run = _oracle_call(w, b, L)
         t0 = time.perf_counter()
-        om.mla_decode(q, kv, np.array([L], np.int32), None, w.softmax_scale, w.causal, q_lens=ql)
+        run(q, np.array([L], np.int32), ql)
         t_total += time.perf_counter() - t0
-        done_bytes += L * 1152
+        done_bytes += L * (580 if w.fp8 else 1152)
         done_flops += W_flops([L], w, ql)
         seqs.append(b)
         if t_total >= target_s:
@@ -258,6 +268,29 @@ def oracle_baseline(w, target_s: float = 12.0):
             "tflops": done_flops / t_total / 1e12,
             "sample": f"{len(seqs)} whole sequence(s) of the workload (index {seqs[0]}..{seqs[-1]}), "
                       f"{done_bytes / 1e9:.3f} GB of KV, fp64 C oracle with OpenMP, {t_total:.2f} s"}
+
+
+def _oracle_call(w, b: int, rows: int):
+    """The oracle on the first `rows` cache rows of sequence b (bf16 or E4M3 cache) as a callable
+    (q_bits, seqlens, q_lens) -> (O, LSE); the cache rows are gathered before it is timed."""
+    from mla_decode_attention_etap_b200.workloads import bf16_bits
+    from oracle import mla_oracle as om
+
+    def seq_rows(t):
+        L = int(w.seqlens[b])
+        if w.block_table is None:
+            out = t[b, :L]
+        else:
+            nb = (L + 63) // 64
+            out = t[w.block_table[b, :nb].long().to(t.device)].reshape(nb * 64, *t.shape[2:])[:L]
+        return out[:rows].cpu()
+
+    if w.fp8:
+        codes = seq_rows(w.kv8).numpy().reshape(1, rows, 576)
+        sc = seq_rows(w.kv_scale).numpy().reshape(1, rows)
+        return lambda q, sl, ql: om.mla_decode_fp8(q, codes, sc, sl, None, w.softmax_scale, w.causal, q_lens=ql)
+    kv = bf16_bits(seq_rows(w.kv).reshape(1, rows, 576))
+    return lambda q, sl, ql: om.mla_decode(q, kv, sl, None, w.softmax_scale, w.causal, q_lens=ql)
 
 
 # ---------------------------------------------------------------- arms
@@ -277,17 +310,17 @@ def run_reference(args):
     # one step = the oracle over a bounded slice of the workload: the first sequence, first 4096 rows
     b = 0
     L = min(int(w.seqlens[b]), args.reference_rows)
-    kv = bf16_bits(w.kv_rows(b)[:L].cpu().reshape(1, L, 576))
+    run = _oracle_call(w, b, L)
     q = bf16_bits(w.q[b:b + 1].cpu())
     sl = np.array([L], np.int32)
     ql = None if w.q_lens is None else w.q_lens[b:b + 1].numpy()
     for _ in range(args.warmup):
-        om.mla_decode(q, kv, sl, None, w.softmax_scale, w.causal, q_lens=ql)
+        run(q, sl, ql)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        om.mla_decode(q, kv, sl, None, w.softmax_scale, w.causal, q_lens=ql)
+        run(q, sl, ql)
     dt = (time.perf_counter() - t0) / args.steps
-    value = L * 1152 / dt / 1e12
+    value = L * (580 if w.fp8 else 1152) / dt / 1e12
     sample = f"sequence 0, first {L} cache rows, all {w.num_heads} heads x {w.q_len} token(s), per step"
     line = {"metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -322,7 +355,10 @@ def run_ours(args):
     o = torch.empty(B, q_len, h, 512, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(B, q_len, h, dtype=torch.float32, device=dev)
     seqlens = [int(x) for x in w.seqlens]
-    kv_bytes = W.algorithmic_kv_bytes(seqlens)
+    fp8 = w.fp8
+    if fp8:
+        kv, kv_scale = w.kv8, w.kv_scale  # the cache the decode reads: E4M3 codes + row scales
+    kv_bytes = W.algorithmic_kv_bytes(seqlens, fp8=fp8)
     q_lens = w.q_lens.to(dev) if w.q_lens is not None else None
     flops = W.algorithmic_flops(seqlens, q_len, h, w.causal, None if w.q_lens is None else w.q_lens.tolist())
     stream = torch.cuda.current_stream()
@@ -330,13 +366,20 @@ def run_ours(args):
     n_events = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_events)]
 
+    def decode(q_, kv_, sl_, bt_, ql_, sc_=None):
+        # the decode kernel merges the split-KV partials itself (no combine launch)
+        if fp8:
+            mla.mla_decode_fwd_fp8(q_, kv_, sc_, sl_, bt_, w.softmax_scale, w.causal, o, lse, dec.workspace,
+                                   dec.n_sms, 0, q_lens=ql_)
+        else:
+            mla.mla_decode_fwd(q_, kv_, sl_, bt_, w.softmax_scale, w.causal, o, lse, dec.workspace, dec.n_sms, 0,
+                               q_lens=ql_)
+
     def step(i=None):
         dec.plan(sl)
         if i is not None:
             ev[i][0].record(stream)
-        # the decode kernel merges the split-KV partials itself (no combine launch)
-        mla.mla_decode_fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o, lse, dec.workspace, dec.n_sms, 0,
-                           q_lens=q_lens)
+        decode(q, kv, sl, bt, q_lens, kv_scale if fp8 else None)
         if i is not None:
             ev[i][1].record(stream)
 
@@ -362,23 +405,25 @@ def run_ours(args):
             step(i)
         torch.cuda.synchronize()
         # attainable read bandwidth of the decode's TMA pattern on this GPU: the streaming probe
-        # (same grid, split, slots and L2 prefetch, no computation) over the same cache tensor
-        kv_flat = kv.reshape(-1, 576)
-        probe_rows = (kv_flat.shape[0] // 128) * 128
-        probe_err = torch.zeros(1, dtype=torch.int32, device=dev)
-        probe_units = dec.n_sms // 2
-        for _ in range(3):
-            mla.mla_stream_probe(kv_flat[:probe_rows], probe_units, probe_err)
-        pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        pe0.record(stream)
-        n_probe = max(3, min(args.steps, 50))
-        for _ in range(n_probe):
-            mla.mla_stream_probe(kv_flat[:probe_rows], probe_units, probe_err)
-        pe1.record(stream)
-        torch.cuda.synchronize()
-        probe_s = pe0.elapsed_time(pe1) / 1e3 / n_probe
-        if int(probe_err.item()) != 0:
-            raise RuntimeError("streaming probe: a bounded wait ran out")
+        # (same grid, split, slots and L2 prefetch, no computation) over the same bf16 cache tensor
+        probe_s = None
+        if not fp8:
+            kv_flat = kv.reshape(-1, 576)
+            probe_rows = (kv_flat.shape[0] // 128) * 128
+            probe_err = torch.zeros(1, dtype=torch.int32, device=dev)
+            probe_units = dec.n_sms // 2
+            for _ in range(3):
+                mla.mla_stream_probe(kv_flat[:probe_rows], probe_units, probe_err)
+            pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            pe0.record(stream)
+            n_probe = max(3, min(args.steps, 50))
+            for _ in range(n_probe):
+                mla.mla_stream_probe(kv_flat[:probe_rows], probe_units, probe_err)
+            pe1.record(stream)
+            torch.cuda.synchronize()
+            probe_s = pe0.elapsed_time(pe1) / 1e3 / n_probe
+            if int(probe_err.item()) != 0:
+                raise RuntimeError("streaming probe: a bounded wait ran out")
     status = dec.status()
     if status != 0:
         raise RuntimeError(f"device status {mla.STATUS.get(status, status)}")
@@ -391,6 +436,8 @@ def run_ours(args):
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     hq = q.cpu().pin_memory()
     hkv = kv.cpu().pin_memory()
+    hsc = kv_scale.cpu().pin_memory() if fp8 else None
+    dsc = torch.empty_like(kv_scale) if fp8 else None
     hsl = w.seqlens.clone().pin_memory()
     hbt = w.block_table.clone().pin_memory() if w.block_table is not None else None
     ho = torch.empty_like(o, device="cpu").pin_memory()
@@ -399,8 +446,9 @@ def run_ours(args):
     dbt = torch.empty_like(bt) if bt is not None else None
     hql = w.q_lens.clone().pin_memory() if w.q_lens is not None else None
     dql = torch.empty_like(q_lens) if q_lens is not None else None
-    h2d = (hq.numel() * 2 + hkv.numel() * 2 + hsl.numel() * 4 + (hbt.numel() * 4 if hbt is not None else 0)
-           + (hql.numel() * 4 if hql is not None else 0))
+    h2d = (hq.numel() * 2 + hkv.numel() * hkv.element_size() + hsl.numel() * 4
+           + (hbt.numel() * 4 if hbt is not None else 0) + (hql.numel() * 4 if hql is not None else 0)
+           + (hsc.numel() * 4 if hsc is not None else 0))
     d2h = ho.numel() * 2 + hl.numel() * 4
 
     def e2e_step():
@@ -411,9 +459,10 @@ def run_ours(args):
             dbt.copy_(hbt, non_blocking=True)
         if dql is not None:
             dql.copy_(hql, non_blocking=True)
+        if dsc is not None:
+            dsc.copy_(hsc, non_blocking=True)
         dec.plan(dsl)
-        mla.mla_decode_fwd(dq, dkv, dsl, dbt, w.softmax_scale, w.causal, o, lse, dec.workspace, dec.n_sms, 0,
-                           q_lens=dql)
+        decode(dq, dkv, dsl, dbt, dql, dsc)
         ho.copy_(o, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
 
@@ -440,11 +489,15 @@ def run_ours(args):
             roof = {"bound": "tensor", "achieved": ach, "peak": tc_tflops, "unit": "TFLOP/s", "frac": ach / tc_tflops}
         roof["traffic"] = profiled_traffic(wname)
         roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
-        roof["attainable_read_gbs"] = probe_rows * 1152 / probe_s / 1e9
-        roof["frac_of_attainable"] = roof["achieved"] / roof["attainable_read_gbs"] if bound == "hbm" else None
-        roof["attainable_note"] = ("streaming probe: the decode's TMA read pattern (same grid, column split, "
-                                   "5 V-pair slots, L2 prefetch) without computation, over the same cache")
-        roof["kernel"] = "etap_pair_kernel"
+        if probe_s is not None:
+            roof["attainable_read_gbs"] = probe_rows * 1152 / probe_s / 1e9
+            roof["frac_of_attainable"] = roof["achieved"] / roof["attainable_read_gbs"] if bound == "hbm" else None
+            roof["attainable_note"] = ("streaming probe: the decode's TMA read pattern (same grid, column split, "
+                                       "5 V-pair slots, L2 prefetch) without computation, over the same cache")
+        else:
+            roof["attainable_read_gbs"] = None
+            roof["attainable_note"] = "no streaming probe for the E4M3 cache's read pattern"
+        roof["kernel"] = "etap_pair_kernel<PairCfg16E4>" if fp8 else "etap_pair_kernel"
         roof["kernel_ms"] = kern_s * 1e3
         roof["kernel_timing"] = ("CUDA events on the launch stream around each of K decode launches, "
                                  "in a second pass of K steps right after the timed region")
@@ -462,7 +515,7 @@ def run_ours(args):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16",
+            "dtype": "e4m3" if fp8 else "bf16",
             "data": "synthetic",
             "tflops": weak_scaling_value(flops, world, step_s_max) / 1e12,
             "config": {"workload": wname, "batch_per_gpu": B, "heads": h, "q_len": q_len,
@@ -470,6 +523,8 @@ def run_ours(args):
                        "seqlens": (seqlens[0] if len(set(seqlens)) == 1 else
                                    f"{min(seqlens)}..{max(seqlens)} (mean {sum(seqlens) / len(seqlens):.0f})"),
                        "d_qk": 576, "d_v": 512, "kv_layout": "paged64" if bt is not None else "contiguous",
+                       "kv_cache": ("E4M3 codes + fp32 scale per row (580 B/token)" if fp8 else
+                                    "bf16 (1152 B/token)"),
                        "causal": bool(w.causal), "kv_bytes_per_gpu": kv_bytes,
                        "l2": ("inputs larger than L2 (no flush)" if kv_bytes > 126e6 else
                               "inputs smaller than L2 (not flushed; numbers are L2-warm)"),

@@ -150,6 +150,29 @@ MLA_API int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *
                           void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream);
 
 /*
+ * Decode over an FP8 latent cache (a storage format next to the pages' bf16
+ * cache: half the bytes per cached token for the HBM-bound decode).  Every cache
+ * row holds 576 OCP E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa
+ * bits; 0x7F/0xFF are NaN) and one fp32 scale; element k of row r stands for
+ * kv_scale[r] * e4m3(kv8[r][k]), and the result is the attention of
+ * mla_decode_fwd over those values (same definition, outputs and tolerances).
+ *   kv8        uint8 codes, laid out like mla_decode_fwd's kv (contiguous
+ *              [batch, kv_rows, 576] or paged [kv_rows / 64, 64, 576]), 16-byte aligned
+ *   kv_scale   fp32, one scale per cache row, indexed like the rows ([batch, kv_rows]
+ *              or [kv_rows / 64, 64]), 4-byte aligned, must not be NULL; a scale must be
+ *              finite and >= 0 (values below 2^-100 count as 2^-100 in the maximum)
+ *   q_lens     as for mla_decode_fwd_ragged, or NULL
+ * Supported for q_len * num_heads <= 16 (else MLA_ERR_UNSUPPORTED).  The kernel
+ * stores Q per query column as two E4M3 terms times a power of two, and P as two
+ * E4M3 terms; the fp32 accumulation, the split-KV merge and the outputs are those
+ * of mla_decode_fwd.  All other arguments, layouts and errors as there.
+ */
+MLA_API int mla_decode_fwd_fp8(const void *q, const void *kv8, const float *kv_scale, const int32_t *seqlens,
+                       const int32_t *q_lens, const int32_t *block_table, int batch, int q_len, int num_heads,
+                       int64_t kv_rows, int max_blocks, float softmax_scale, int causal, void *o, float *lse,
+                       void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream);
+
+/*
  * Log-sum-exp merge of the split-KV partials that mla_decode_fwd left in the
  * workspace: lse = ln sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s, for
  * every sequence split over several CTAs; also writes O = 0, LSE = -inf for

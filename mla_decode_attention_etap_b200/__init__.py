@@ -28,7 +28,7 @@ STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3:
 
 EXPORTS = ("mla_decode_workspace_size", "mla_decode_plan", "mla_decode_fwd", "mla_combine",
            "mla_decode_read_status", "mla_decode_plan_host", "mla_status_string", "mla_last_cuda_error",
-           "mla_decode_fwd_static_ws", "mla_decode_fwd_ragged", "mla_stream_probe")
+           "mla_decode_fwd_static_ws", "mla_decode_fwd_ragged", "mla_stream_probe", "mla_decode_fwd_fp8")
 STATIC_WORKSPACE_BYTES = 8388608
 
 
@@ -60,6 +60,9 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_fwd_ragged.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp, vp,
                                             vp, sz, i32, ctypes.c_uint, vp]
         L.mla_decode_fwd_ragged.restype = i32
+        L.mla_decode_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp,
+                                         vp, vp, sz, i32, ctypes.c_uint, vp]
+        L.mla_decode_fwd_fp8.restype = i32
         L.mla_combine.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
         L.mla_combine.restype = i32
         L.mla_decode_read_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
@@ -136,6 +139,23 @@ def mla_decode_fwd(q, kv, seqlens, block_table, softmax_scale, causal, o, lse, w
                                            _stream(stream)), "mla_decode_fwd_ragged")
 
 
+def mla_decode_fwd_fp8(q, kv8, kv_scale, seqlens, block_table, softmax_scale, causal, o, lse, workspace, n_sms,
+                       flags=0, stream=None, q_lens=None) -> None:
+    """Decode over an FP8 cache: ``kv8`` uint8 E4M3 codes laid out like the bf16 cache, ``kv_scale``
+    fp32 with one scale per cache row (``mla_decode_fwd_fp8``; h * q_len <= 16)."""
+    B, q_len, h, _ = q.shape
+    if block_table is not None:
+        kv_rows, max_blocks = kv8.shape[0] * kv8.shape[1], block_table.shape[1]
+    else:
+        kv_rows, max_blocks = kv8.shape[1], 0
+    assert kv8.dtype == torch.uint8 and kv_scale.dtype == torch.float32
+    _check(lib().mla_decode_fwd_fp8(_ptr(q), _ptr(kv8), _ptr(kv_scale), _ptr(seqlens), _ptr(q_lens),
+                                    _ptr(block_table), B, q_len, h, kv_rows, max_blocks, float(softmax_scale),
+                                    int(bool(causal)), _ptr(o), _ptr(lse), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), n_sms, flags, _stream(stream)),
+           "mla_decode_fwd_fp8")
+
+
 def mla_stream_probe(kv, units: int, err, stream=None) -> None:
     """Stream ``kv`` ([..., 576] bf16, rows a multiple of 128) with the decode's TMA read pattern and
     no computation (a bandwidth probe).  ``err``: int32 device tensor [1], zeroed by the caller."""
@@ -193,6 +213,19 @@ class MlaDecoder:
         scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(D_QK)
         mla_decode_fwd(q, kv, seqlens, block_table, scale, causal, o, lse, self.workspace, self.n_sms, flags,
                        stream, q_lens=q_lens)
+        return o, lse
+
+    def fwd_fp8(self, q, kv8, kv_scale, seqlens, block_table=None, softmax_scale=None, causal=False, o=None,
+                lse=None, flags=0, stream=None, q_lens=None):
+        """fwd over an FP8 cache (E4M3 codes + one fp32 scale per cache row)."""
+        B, q_len, h, _ = q.shape
+        if o is None:
+            o = torch.empty(B, q_len, h, D_V, dtype=torch.bfloat16, device=q.device)
+        if lse is None:
+            lse = torch.empty(B, q_len, h, dtype=torch.float32, device=q.device)
+        scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(D_QK)
+        mla_decode_fwd_fp8(q, kv8, kv_scale, seqlens, block_table, scale, causal, o, lse, self.workspace, self.n_sms,
+                           flags, stream, q_lens=q_lens)
         return o, lse
 
     def status(self, stream=None) -> int:

@@ -24,6 +24,13 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: p = 2^(x - m) stays <=
 // bf16 hi + lo split keep their relative precision there, and only rows more than ~100 octaves
 // below the maximum underflow to 0, as they would in any fp32 softmax.
 constexpr float kRescaleHeadroom = 24.0f;
+// E4M3 cache: P is stored as two E4M3 terms, whose absolute resolution is fixed (2^-9 at the
+// bottom of the subnormal range), so p must stay close to the maximum: the running maximum is
+// reset to 2 above the tile maximum and moves once a row exceeds it by 4, and p is stored times
+// 2^4 (at most 2^8, inside the E4M3 range of 448).
+constexpr float kRescaleThreshold8 = 4.0f;
+constexpr float kRescaleHeadroom8 = 2.0f;
+constexpr float kPScaleLog2_8 = 4.0f;
 
 // Per-CTA wait control in shared memory: the abort flag every role polls and
 // the bound after which a wait gives up.
@@ -34,6 +41,8 @@ struct WaitCtl {
 };
 
 struct DecodeParams {
+    const __nv_bfloat16 *q;   // [B, q_len, h, 576] (read directly only by the E4M3-cache kernel)
+    const float *kv_scale;    // E4M3 cache: one fp32 scale per cache row, indexed like the rows
     const int32_t *seqlens;
     const int32_t *q_lens;  // ragged batch: query tokens per sequence (<= q_len), or NULL
     const int32_t *block_table;
@@ -113,28 +122,42 @@ struct SegIter {
 };
 
 // Tile-by-tile cursor over the same segments (the MMA issuer keeps one for
-// the scores and one for the output contraction).
-struct TileCursor {
+// the scores and one for the output contraction).  STEP > 1: only tiles
+// t0 + off, t0 + off + STEP, ... of each segment, skipping segments that have none.
+template <int STEP = 1>
+struct TileCursorT {
     SegIter it;
-    int b, t0, t, t1;
+    int b, t0, t, t1, off;
     bool valid;
-    __device__ void init(const int32_t *tile_off, int batch, int64_t fb, int64_t fe) {
+    __device__ void skip_empty(const int32_t *tile_off) {
+        if constexpr (STEP > 1) {
+            while (valid && t >= t1) {
+                valid = it.next(tile_off, b, t0, t1);
+                t = t0 + off;
+            }
+        }
+    }
+    __device__ void init(const int32_t *tile_off, int batch, int64_t fb, int64_t fe, int off_ = 0) {
         it.init(tile_off, batch, fb, fe);
+        off = STEP > 1 ? off_ : 0;
         b = t0 = t = t1 = 0;
         valid = it.next(tile_off, b, t0, t1);
-        t = t0;
+        t = t0 + off;
+        skip_empty(tile_off);
     }
     __device__ void advance(const int32_t *tile_off) {
-        if (t + 1 < t1) {
-            ++t;
+        if (t + STEP < t1) {
+            t += STEP;
             return;
         }
         valid = it.next(tile_off, b, t0, t1);
-        t = t0;
+        t = t0 + off;
+        skip_empty(tile_off);
     }
-    __device__ bool first() const { return t == t0; }
-    __device__ bool last() const { return t == t1 - 1; }
+    __device__ bool first() const { return t == t0 + off; }
+    __device__ bool last() const { return t + STEP >= t1; }
 };
+using TileCursor = TileCursorT<1>;
 
 // Column reduction of 16 values per lane across the 32 lanes of a warp
 // (recursive halving: 16 shuffles instead of 5 per column).  Lane l ends with

@@ -43,64 +43,98 @@ __host__ __device__ constexpr uint32_t pow2_at_least(uint32_t x) {
     return x <= 32 ? 32 : x <= 64 ? 64 : x <= 128 ? 128 : x <= 256 ? 256 : 512;
 }
 
-// NG query columns per cluster; NV V-pair slots, NR rope slots, PB P^T buffers per CTA.
-template <int NG_, int NV_, int NR_, int PB_>
+// NG query columns per cluster; NV V slots, NR rope slots, PB P^T buffers per CTA.
+//
+// KV8: the cache holds E4M3 codes plus one fp32 scale per row, and both contractions run as
+// kind::f8f6f4 MMAs (Q and P each split into two E4M3 terms).  A whole 576-code tile then takes
+// the shared memory a bf16 half tile takes, so the two CTAs of a cluster do not split tiles by
+// columns: each takes every other tile of the pair's range with all 576 columns (no per-tile
+// score exchange) and the two partial results of a segment are merged once, at its end,
+// through distributed shared memory.
+template <int NG_, int NV_, int NR_, int PB_, bool KV8_ = false>
 struct PairCfg {
+    static constexpr bool KV8 = KV8_;
     static constexpr int NG = NG_;
-    static constexpr int NP = 2 * NG;  // UMMA N of step 3: [P_hi | P_lo]
+    static constexpr int NP = 2 * NG;             // UMMA N of step 3: [P_hi | P_lo]
+    static constexpr int NS = KV8 ? 2 * NG : NG;  // UMMA N of step 1 (E4M3: [Q_hi | Q_lo] products)
     static constexpr int CH = NG / 16;  // 16-column chunks of softmax and exchange
     static constexpr int NV = NV_, NR = NR_, PB = PB_;
-    static constexpr int PAIRS = 2;                                    // V pairs of a tile in one CTA
-    static constexpr int EARLY = (NV - PAIRS) < PAIRS ? (NV - PAIRS) : PAIRS;  // pairs of tile k+1 free of tile k
+    // V slots of a tile in one CTA: a slot is two 128-row chunks of 128 bytes per row
+    // (bf16: 2 x 64 latent columns, a "V pair"; E4M3: 2 x 128, the CTA's whole V half)
+    static constexpr int PAIRS = 2;
+    static constexpr int MB = KV8 ? 4 : 2;        // M-tiles of O^T (128 latent rows each) per CTA
+    static constexpr int TSTEP = KV8 ? 2 : 1;     // tiles of a segment taken by one CTA: every TSTEP-th
+    static constexpr int CHUNK_COLS = KV8 ? 128 : 64;
+    static constexpr int VCOLS = KV8 ? 512 : 256;  // latent (V) columns of a tile this CTA loads
     static constexpr int XS = CH > 2 ? CH : 2;                         // exchange slots (8 KB each)
+    // KV8: the segment merge receives 2 M-tiles x 128 rows x 16 fp32 plus 16 (m, l) per softmax warp
+    static constexpr uint32_t X_BYTES = KV8 ? 2 * 128 * 16 * 4 + 8 * 16 * 4 : XS * 128 * 16 * 4;
     // One column chunk per thread (h*q_len <= 16): the softmax warps issue step 3 themselves, right
     // after the barrier that ends the tile, instead of handing P^T to the MMA warp (its polling and
     // the score MMAs it may be issuing would delay it); the issuing warp has a tile's time to spare.
     static constexpr bool PV_BY_SOFTMAX = CH == 1;
     static constexpr int PREFETCH = 1;                                 // tiles the L2 prefetch runs ahead of the loads
-    static constexpr uint32_t CHUNK = 16384;                           // 128 rows x 64 bf16, 128B swizzle
+    static constexpr uint32_t CHUNK = 16384;                           // 128 rows x 128 bytes, 128B swizzle
     static constexpr uint32_t HALF = 8192;                             // 64 rows of a chunk = one TMA box
     static constexpr uint32_t V_SLOT = 2 * CHUNK;
-    static constexpr uint32_t R_SLOT = 128 * 64;                       // 128 rows x 32 rope bf16, 64B swizzle
-    static constexpr uint32_t R_HALF = 64 * 64;                        // 64 rows of it = one TMA box
-    static constexpr uint32_t Q_CHUNK = NG * 128;                      // NG rows x 64 columns
-    static constexpr uint32_t Q_ROPE = NG * 64;                        // NG rows x 32 rope columns
-    static constexpr int AW = NP < 64 ? NP : 64;                       // P^T swizzle atom width (columns)
+    // bytes of a row's rope codes in this CTA: bf16 32 columns (its half), E4M3 all 64
+    static constexpr uint32_t R_ROW = 64;
+    static constexpr uint32_t R_DATA = 128 * R_ROW;
+    // E4M3: the rope slot also receives the tile's 128 row scales
+    static constexpr uint32_t R_SLOT = KV8 ? align1024(R_DATA + 128 * 4) : R_DATA;
+    static constexpr uint32_t R_HALF = 64 * R_ROW;                     // 64 rows of it = one TMA box
+    static constexpr uint32_t R_SWIZZLE = kSwizzle64B;
+    static constexpr int R_KSTEPS = 2;                                 // 32-byte K-steps over the rope
+    static constexpr int QROWS = KV8 ? 2 * NG : NG;                    // B operand rows of step 1
+    static constexpr int Q_CHUNKS = 4;                                 // 128-byte chunks of the V columns
+    static constexpr uint32_t Q_CHUNK = QROWS * 128;
+    static constexpr uint32_t Q_ROPE = QROWS * R_ROW;
+    static constexpr int PE = KV8 ? 1 : 2;                             // bytes per P^T element
+    static constexpr uint32_t P_PITCH = NP * PE < 128 ? NP * PE : 128; // bytes per KV row inside an atom
+    static constexpr int AW = P_PITCH / PE;                            // P^T swizzle atom width (columns)
     static constexpr int NA = NP / AW;                                 // atoms along N
-    static constexpr uint32_t P_PITCH = AW * 2;                        // bytes per KV row inside an atom
     static constexpr uint32_t P_ATOM = 128 * P_PITCH;
     static constexpr uint32_t P_BUF = NA * P_ATOM;
-    static constexpr uint32_t P_SWIZZLE = (P_PITCH == 128) ? kSwizzle128B : kSwizzle64B;
-    static constexpr uint32_t P_SWZ_MASK = (P_PITCH == 128) ? 7u : 3u;
+    static constexpr uint32_t P_SWIZZLE = P_PITCH == 128 ? kSwizzle128B : P_PITCH == 64 ? kSwizzle64B : kSwizzle32B;
+    static constexpr uint32_t P_SWZ_MASK = P_PITCH == 128 ? 7u : P_PITCH == 64 ? 3u : 1u;
+    static constexpr int P_ROWS_MMA = KV8 ? 32 : 16;                   // KV rows (K) per step-3 MMA
     static constexpr uint32_t X_SLOT = 128 * 16 * 4;                   // 128 rows x 16 fp32 partial scores
     static constexpr uint32_t OFF_V = 0;
     static constexpr uint32_t OFF_R = OFF_V + NV * V_SLOT;
     static constexpr uint32_t OFF_Q = OFF_R + NR * R_SLOT;
-    static constexpr uint32_t OFF_QR = OFF_Q + 4 * Q_CHUNK;
+    static constexpr uint32_t OFF_QR = OFF_Q + Q_CHUNKS * Q_CHUNK;
     static constexpr uint32_t OFF_P = align1024(OFF_QR + Q_ROPE);
     static constexpr uint32_t OFF_X = OFF_P + PB * P_BUF;
-    static constexpr uint32_t OFF_BAR = OFF_X + XS * X_SLOT;
+    static constexpr uint32_t OFF_BAR = OFF_X + X_BYTES;
     static constexpr uint32_t OFF_RED = OFF_BAR + 512;                 // float [2][4][NG] column max exchange
     static constexpr uint32_t OFF_REDL = OFF_RED + 32 * NG;               // float [4][NG] column sum exchange
-    static constexpr uint32_t OFF_MISC = OFF_REDL + 16 * NG;
+    static constexpr uint32_t OFF_QSC = OFF_REDL + 16 * NG;            // E4M3: float [2][NG] Q column factors
+    static constexpr uint32_t OFF_MISC = OFF_QSC + 8 * NG;
     static constexpr uint32_t BYTES = OFF_MISC + 64;
     static constexpr uint32_t SMEM_ALLOC = BYTES + 1024;               // slack for 1024-byte alignment
-    static constexpr uint32_t O_COL = 0;                               // 2 M-tiles x NP columns
-    static constexpr uint32_t S_COL = 2 * NP;                          // 2 buffers x NG columns
-    static constexpr uint32_t TMEM_COLS = pow2_at_least(2 * NP + 2 * NG);
-    static constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, NG, 0, 0);
-    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, NP, 1, 1);
+    static constexpr uint32_t O_COL = 0;                               // MB M-tiles x NP columns
+    static constexpr uint32_t S_COL = MB * NP;                         // 2 buffers x NS columns
+    static constexpr uint32_t TMEM_COLS = pow2_at_least(MB * NP + 2 * NS);
+    static constexpr uint32_t IDESC_QK = KV8 ? idesc_e4m3_f32(128, NS, 0, 0) : idesc_bf16_f32(128, NG, 0, 0);
+    static constexpr uint32_t IDESC_PV = KV8 ? idesc_e4m3_f32(128, NP, 1, 1) : idesc_bf16_f32(128, NP, 1, 1);
+    static constexpr float THRESH = KV8 ? kRescaleThreshold8 : kRescaleThreshold;
+    static constexpr float HEADROOM = KV8 ? kRescaleHeadroom8 : kRescaleHeadroom;
     // The in-kernel split merge stages (splits + 1) x NG floats in the idle P^T buffers.
     static constexpr int MERGE_MAX_SPLITS = (int)(PB * P_BUF / 4) / NG - 1;
 };
 
 using PairCfg16 = PairCfg<16, 5, 2, 2>;  // h*q_len <= 16
 using PairCfg32 = PairCfg<32, 5, 1, 1>;  // 16 < h*q_len, in groups of 32 columns
+// E4M3 cache, h*q_len <= 16: whole tiles per CTA, 2.5 tiles in flight
+using PairCfg16E4 = PairCfg<16, 5, 2, 2, true>;
 
-static_assert(PairCfg16::SMEM_ALLOC <= 232448 && PairCfg32::SMEM_ALLOC <= 232448, "shared memory plan > 227 KB");
-static_assert(PairCfg16::TMEM_COLS <= 512 && PairCfg32::TMEM_COLS <= 512, "TMEM plan");
-static_assert(PairCfg16::OFF_P % 1024 == 0 && PairCfg32::OFF_P % 1024 == 0, "alignment");
-static_assert(PairCfg16::OFF_QR % 512 == 0 && PairCfg32::OFF_QR % 512 == 0, "alignment");
+template <class C>
+constexpr bool pair_cfg_fits() {
+    return C::SMEM_ALLOC <= 232448 && C::TMEM_COLS <= 512 && C::OFF_P % 1024 == 0 && C::OFF_QR % 512 == 0 &&
+           C::OFF_R % 1024 == 0 && C::R_SLOT % 256 == 0 && C::OFF_Q % 1024 == 0 && (!C::KV8 || C::CH == 1);
+}
+static_assert(pair_cfg_fits<PairCfg16>() && pair_cfg_fits<PairCfg32>() && pair_cfg_fits<PairCfg16E4>(),
+              "shared memory / TMEM plan");
 
 template <class C>
 struct PairBars {
@@ -126,7 +160,9 @@ struct PairBars {
     static constexpr int XFREE = XFULL + 8 * C::XS;  // [8], used when CH > 1: the peer consumed our last tile
     static constexpr int COUNT = XFREE + 8;
 };
-static_assert(PairBars<PairCfg16>::COUNT * 8 <= 512 && PairBars<PairCfg32>::COUNT * 8 <= 512, "barrier area");
+static_assert(PairBars<PairCfg16>::COUNT * 8 <= 512 && PairBars<PairCfg32>::COUNT * 8 <= 512 &&
+                  PairBars<PairCfg16E4>::COUNT * 8 <= 512,
+              "barrier area");
 
 // Byte offset of 16-byte chunk j of row r in a row-major buffer of `pitch`-byte
 // rows swizzled like the MMA operand (chunk index XOR address bits 7+).
@@ -166,10 +202,13 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(bar(BR::VEMPTY + i), 1);
         }
         for (int i = 0; i < C::NR; ++i) {
-            mbar_init(bar(BR::RFULL + i), 1);
-            mbar_init(bar(BR::REMPTY + i), 1);
+            // E4M3: the rope TMA (one arrival) and the 32 producer lanes' row-scale copies; the slot
+            // is freed by the 8 softmax warps once they have read the scales
+            mbar_init(bar(BR::RFULL + i), C::KV8 ? 33 : 1);
+            mbar_init(bar(BR::REMPTY + i), C::KV8 ? 8 : 1);
         }
-        mbar_init(bar(BR::QFULL), 1);
+        // E4M3: the softmax warps write the quantised Q operand themselves
+        mbar_init(bar(BR::QFULL), C::KV8 ? 8 : 1);
         mbar_init(bar(BR::QEMPTY), 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(BR::SFULL + i), 1);
@@ -191,9 +230,11 @@ __global__ void __launch_bounds__(320, 1)
         fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tm_q);
+        if constexpr (!C::KV8) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_qr);
+        }
         tma_prefetch_desc(&tm_kv);
-        tma_prefetch_desc(&tm_qr);
         tma_prefetch_desc(&tm_kvr);
     }
     if (warp == 1) {
@@ -204,8 +245,8 @@ __global__ void __launch_bounds__(320, 1)
     cluster_sync();  // both CTAs' barriers are initialised before any remote arrive or st.async
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // Step 3 of tile kk: O^T (+)= V^T P^T for both V pairs of this CTA; frees each V slot and then
-    // the P^T buffer as the MMAs complete.
+    // Step 3 of tile kk: O^T (+)= V^T P^T for the CTA's 256 latent rows (two M-tiles); frees each
+    // V slot and then the P^T buffer as the MMAs complete.
     auto issue_pv = [&](int kk, bool first) {
         const int pb = kk % C::PB;
         const uint32_t p_base = sbase + C::OFF_P + pb * C::P_BUF;
@@ -213,14 +254,32 @@ __global__ void __launch_bounds__(320, 1)
             const int g2 = C::PAIRS * kk + i;
             const int vs = g2 % C::NV;
             const uint32_t v_base = sbase + C::OFF_V + vs * C::V_SLOT;
-            const uint32_t d_o = tmem + C::O_COL + i * C::NP;
+            if constexpr (C::KV8) {
+                // slot i = M-tiles 2i, 2i+1: chunk mt of the slot holds latent columns 256 i + 128 mt..
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                // A = V^T: M = 128 latent columns (two chunks CHUNK apart), K = 16 KV rows (MN-major)
-                const uint64_t a = smem_desc(v_base + 2048u * s, C::CHUNK, 1024, kSwizzle128B);
-                // B = [P_hi | P_lo]^T: K = 16 KV rows, N = NP columns (MN-major)
-                const uint64_t bp = smem_desc(p_base + 16u * C::P_PITCH * s, C::P_ATOM, 8 * C::P_PITCH, C::P_SWIZZLE);
-                umma_bf16(d_o, a, bp, C::IDESC_PV, (first && s == 0) ? 0u : 1u);
+                for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+                    for (int s = 0; s < 128 / C::P_ROWS_MMA; ++s) {
+                        // A = V^T: M = 128 latent columns (one 128-byte swizzle row), K = 32 KV rows (MN-major)
+                        const uint64_t a = smem_desc(v_base + mt * C::CHUNK + 4096u * s, C::CHUNK, 1024, kSwizzle128B);
+                        // B = [P_hi | P_lo]^T: K = 32 KV rows, N = NP columns (MN-major)
+                        const uint64_t bp = smem_desc(p_base + 32u * C::P_PITCH * s, C::P_ATOM, 8 * C::P_PITCH,
+                                                      C::P_SWIZZLE);
+                        umma_e4m3(tmem + C::O_COL + (2 * i + mt) * C::NP, a, bp, C::IDESC_PV,
+                                  (first && s == 0) ? 0u : 1u);
+                    }
+                }
+            } else {
+                const uint32_t d_o = tmem + C::O_COL + i * C::NP;
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    // A = V^T: M = 128 latent columns (two chunks CHUNK apart), K = 16 KV rows (MN-major)
+                    const uint64_t a = smem_desc(v_base + 2048u * s, C::CHUNK, 1024, kSwizzle128B);
+                    // B = [P_hi | P_lo]^T: K = 16 KV rows, N = NP columns (MN-major)
+                    const uint64_t bp =
+                        smem_desc(p_base + 16u * C::P_PITCH * s, C::P_ATOM, 8 * C::P_PITCH, C::P_SWIZZLE);
+                    umma_bf16(d_o, a, bp, C::IDESC_PV, (first && s == 0) ? 0u : 1u);
+                }
             }
             umma_commit(bar(BR::VEMPTY + vs));
         }
@@ -242,7 +301,10 @@ __global__ void __launch_bounds__(320, 1)
     const int64_t fb = plan_ok ? ranges[2 * unit] : 0, fe = plan_ok ? ranges[2 * unit + 1] : 0;
     if (!plan_ok && threadIdx.x == 0) atomicCAS(status, 0, kStatusInvalid);
     const int64_t l_cap = p.paged ? (int64_t)p.max_blocks * kPage : p.kv_rows;
-    const int rope_x = 512 + 32 * (int)rank;  // first rope column of this CTA
+    // first rope column of this CTA (E4M3: all 64 rope columns, every CTA)
+    const int rope_x = C::KV8 ? 512 : 512 + 32 * (int)rank;
+    const int kv_x0 = C::KV8 ? 0 : 256 * (int)rank;  // first latent column of this CTA
+    const int toff = C::KV8 ? (int)rank : 0;        // first tile of a segment this CTA takes
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -273,13 +335,14 @@ __global__ void __launch_bounds__(320, 1)
                 } else {
                     yp = (int)((int64_t)pb_ * p.kv_rows + r0 + 64 * hh);
                 }
-                for (int c = 0; c < 4; ++c) tma_prefetch_l2_2d(&tm_kv, (4 * (int)rank + c) * 64, yp);
+                for (int c = 0; c < C::VCOLS / C::CHUNK_COLS; ++c)
+                    tma_prefetch_l2_2d(&tm_kv, kv_x0 + C::CHUNK_COLS * c, yp);
                 tma_prefetch_l2_2d(&tm_kvr, rope_x, yp);
             }
         };
-        TileCursor ahead;
+        TileCursorT<C::TSTEP> ahead;
         if (fb < fe && lane == 0) {
-            ahead.init(tile_off, p.batch, fb, fe);
+            ahead.init(tile_off, p.batch, fb, fe, toff);
             for (int d = 0; d < C::PREFETCH && ahead.valid; ++d) {
                 prefetch_tile(ahead.b, ahead.t);
                 ahead.advance(tile_off);
@@ -296,9 +359,9 @@ __global__ void __launch_bounds__(320, 1)
                     L = (int)l_cap;
                 }
                 if (L < 0) L = 0;
-                if (seg > 0) ok = wait_phase(bar(BR::QEMPTY), (seg - 1) & 1, wc, status);
+                if (!C::KV8 && seg > 0) ok = wait_phase(bar(BR::QEMPTY), (seg - 1) & 1, wc, status);
                 if (!ok) break;
-                if (lane == 0 && !p.withhold_q) {
+                if (!C::KV8 && lane == 0 && !p.withhold_q) {
                     mbar_arrive_expect_tx(bar(BR::QFULL), 4 * C::Q_CHUNK + C::Q_ROPE);
                     const int qrow = b * p.ncols + grp * NG;
                     for (int j = 0; j < 4; ++j)
@@ -306,8 +369,8 @@ __global__ void __launch_bounds__(320, 1)
                                     qrow);
                     tma_load_2d(sbase + C::OFF_QR, &tm_qr, bar(BR::QFULL), rope_x, qrow);
                 }
-                if (!p.withhold_q) ++arms_q;
-                for (int t = t0; t < t1 && ok; ++t, ++k) {
+                if (!C::KV8 && !p.withhold_q) ++arms_q;
+                for (int t = t0 + toff; t < t1 && ok; t += C::TSTEP, ++k) {
                     if (lane == 0 && ahead.valid) {
                         prefetch_tile(ahead.b, ahead.t);
                         ahead.advance(tile_off);
@@ -349,12 +412,23 @@ __global__ void __launch_bounds__(320, 1)
                                     tma_load_2d(sbase + C::OFF_R + rs * C::R_SLOT + hh * C::R_HALF, &tm_kvr,
                                                 bar(BR::RFULL + rs), rope_x, y[hh]);
                         }
+                        if constexpr (C::KV8) {
+                            // the tile's row scales behind the rope codes: lane l copies rows 4l..4l+3
+                            const uint32_t sdst = sbase + C::OFF_R + rs * C::R_SLOT + C::R_DATA;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int r = 4 * lane + u;
+                                if (r < valid && loaded[r >> 6])
+                                    cp_async4(sdst + 4u * r, p.kv_scale + (int64_t)y[r >> 6] + (r & 63));
+                            }
+                            cp_async_mbar_arrive(bar(BR::RFULL + rs));
+                        }
                         ++arms_r[rs];
                     }
                     for (int i = 0; i < C::PAIRS && ok; ++i) {
                         const int g2 = C::PAIRS * k + i;
                         const int vs = g2 % C::NV;
-                        const int c0 = 4 * (int)rank + 2 * i;  // latent chunks c0, c0+1 of this CTA's half
+                        const int x0 = kv_x0 + C::CHUNK_COLS * 2 * i;  // first latent column of the slot
                         ok = wait_phase(bar(BR::VEMPTY + vs), ((g2 / C::NV) & 1) ^ 1, wc, status);
                         if (!ok) break;
                         const uint32_t dst = sbase + C::OFF_V + vs * C::V_SLOT;
@@ -364,7 +438,7 @@ __global__ void __launch_bounds__(320, 1)
                                 for (int hc = 0; hc < 2; ++hc)
                                     for (int hh = 0; hh < 2; ++hh)
                                         tma_load_2d(dst + hc * C::CHUNK + hh * C::HALF, &tm_kv, bar(BR::VFULL + vs),
-                                                    (c0 + hc) * 64, y[hh]);
+                                                    x0 + C::CHUNK_COLS * hc, y[hh]);
                             }
                             ++phases_v[vs];
                             tma_v[vs] = true;
@@ -378,7 +452,7 @@ __global__ void __launch_bounds__(320, 1)
                                         for (int hh = 0; hh < 2; ++hh)
                                             if (loaded[hh])
                                                 tma_load_2d(dst + hc * C::CHUNK + hh * C::HALF, &tm_kv, bar(BR::TAIL),
-                                                            (c0 + hc) * 64, y[hh]);
+                                                            x0 + C::CHUNK_COLS * hc, y[hh]);
                                 }
                                 ok = wait_phase(bar(BR::TAIL), tail_uses & 1, wc, status);
                                 ++tail_uses;
@@ -421,17 +495,21 @@ __global__ void __launch_bounds__(320, 1)
         // tile k-1 on the tensor pipe.
         if (lane == 0 && fb < fe) {
             const uint32_t q_base = sbase + C::OFF_Q;
+            // one 128-byte chunk of K-major operands: four 32-byte K-steps (16 bf16 or 32 E4M3)
             auto qk_chunk = [&](uint32_t d_s, uint32_t a_base, int qchunk, bool init) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const uint64_t a = smem_desc(a_base + 32u * j, 16, 1024, kSwizzle128B);
                     const uint64_t bq = smem_desc(q_base + qchunk * C::Q_CHUNK + 32u * j, 16, 1024, kSwizzle128B);
-                    umma_bf16(d_s, a, bq, C::IDESC_QK, (init && j == 0) ? 0u : 1u);
+                    if constexpr (C::KV8)
+                        umma_e4m3(d_s, a, bq, C::IDESC_QK, (init && j == 0) ? 0u : 1u);
+                    else
+                        umma_bf16(d_s, a, bq, C::IDESC_QK, (init && j == 0) ? 0u : 1u);
                 }
             };
-            TileCursor qc, pc;
-            qc.init(tile_off, p.batch, fb, fe);
-            pc.init(tile_off, p.batch, fb, fe);
+            TileCursorT<C::TSTEP> qc, pc;
+            qc.init(tile_off, p.batch, fb, fe, toff);
+            pc.init(tile_off, p.batch, fb, fe, toff);
             int kq = 0, kp = 0, seg_q = 0;
             int qstage = 0;  // scores of tile kq: 0 = rope columns next, 1 + i = V pair i next
             uint64_t t_last = global_timer_ns();
@@ -449,7 +527,7 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 // step 1 in stages, each as soon as its operands have landed
                 if (qc.valid) {
-                    const uint32_t d_s = tmem + C::S_COL + (kq & 1) * NG;
+                    const uint32_t d_s = tmem + C::S_COL + (kq & 1) * C::NS;
                     if (qstage == 0) {
                         const int rs = kq % C::NR;
                         bool ready = mbar_test_wait(bar(BR::SEMPTY + (kq & 1)), ((kq >> 1) & 1) ^ 1);
@@ -457,15 +535,21 @@ __global__ void __launch_bounds__(320, 1)
                         if (ready) ready = mbar_test_wait(bar(BR::RFULL + rs), (kq / C::NR) & 1);
                         if (ready) {
                             tc_fence_after();
-                            // 32 rope columns (K-major, 64-byte rows): two K-steps; the first (re)initialises S^T
+                            // 32 rope columns (K-major rows of R_ROW bytes): 32-byte K-steps; the first
+                            // (re)initialises S^T
 #pragma unroll
-                            for (int j = 0; j < 2; ++j) {
-                                const uint64_t a =
-                                    smem_desc(sbase + C::OFF_R + rs * C::R_SLOT + 32u * j, 16, 512, kSwizzle64B);
-                                const uint64_t bq = smem_desc(sbase + C::OFF_QR + 32u * j, 16, 512, kSwizzle64B);
-                                umma_bf16(d_s, a, bq, C::IDESC_QK, j == 0 ? 0u : 1u);
+                            for (int j = 0; j < C::R_KSTEPS; ++j) {
+                                const uint64_t a = smem_desc(sbase + C::OFF_R + rs * C::R_SLOT + 32u * j, 16,
+                                                             8 * C::R_ROW, C::R_SWIZZLE);
+                                const uint64_t bq =
+                                    smem_desc(sbase + C::OFF_QR + 32u * j, 16, 8 * C::R_ROW, C::R_SWIZZLE);
+                                if constexpr (C::KV8)
+                                    umma_e4m3(d_s, a, bq, C::IDESC_QK, j == 0 ? 0u : 1u);
+                                else
+                                    umma_bf16(d_s, a, bq, C::IDESC_QK, j == 0 ? 0u : 1u);
                             }
-                            umma_commit(bar(BR::REMPTY + rs));
+                            // E4M3: the softmax warps free the slot after reading its row scales
+                            if constexpr (!C::KV8) umma_commit(bar(BR::REMPTY + rs));
                             qstage = 1;
                             progressed = true;
                         }
@@ -550,7 +634,10 @@ __global__ void __launch_bounds__(320, 1)
             SegIter it;
             it.init(tile_off, p.batch, fb, fe);
             int b, t0, t1, k = 0, seg = 0, e = 0, red_uses = 0;
+            int qseg = 0;  // E4M3: segments with a tile for this CTA (Q operands written so far)
+            int mseg = 0;  // E4M3: segment merges with the peer so far
             while (!stop && it.next(tile_off, b, t0, t1)) {
+                const bool has_tiles = t0 + toff < t1;  // E4M3: the peer may hold the only tile
                 int L = p.seqlens[b];
                 if ((int64_t)L > l_cap) L = (int)l_cap;
                 if (L < 0) L = 0;
@@ -585,12 +672,117 @@ __global__ void __launch_bounds__(320, 1)
                     m[n] = -INFINITY;
                     lpart[n] = 0.f;
                 }
-                for (int t = t0; t < t1 && !stop; ++t, ++k) {
-                    const bool first = (t == t0);
+                float qv[NH];  // E4M3: 2^-c of this thread's columns (their Q codes hold q * 2^c)
+                if constexpr (C::KV8) {
+                    // ---- step 1's B operand for this segment: E4M3 codes [Q_hi ; Q_lo] of all 576 columns,
+                    //      query column n scaled by 2^c_n with 128 < max|q_n| 2^c_n <= 256 (Q_lo holds the
+                    //      rounding residual of Q_hi, so that Q_hi + Q_lo keeps the 8 bits of bf16)
+                    float *qsc = reinterpret_cast<float *>(smem + C::OFF_QSC);  // [NG] 2^c, then [NG] 2^-c
+                    const int tid = (warp - 2) * 32 + lane;
+                    if (has_tiles) {
+                        if (qseg > 0) ok = ok && spin_phase<false>(bar(BR::QEMPTY), (qseg - 1) & 1, wc, status);
+                        {
+                            const int n = tid >> 4, part = tid & 15;  // 16 threads per column, 36 values each
+                            const int ng = grp * NG + n;
+                            float amax = 0.f;
+                            if (ng < p.ncols) {
+                                const uint32_t *qw =
+                                    reinterpret_cast<const uint32_t *>(p.q + ((int64_t)b * p.ncols + ng) * kDqk) +
+                                    18 * part;
+#pragma unroll 6
+                                for (int i = 0; i < 18; ++i) {
+                                    const uint32_t w2 = __ldg(qw + i);
+                                    amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w2 << 16)),
+                                                             fabsf(__uint_as_float(w2 & 0xFFFF0000u))));
+                                }
+                            }
+#pragma unroll
+                            for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                            int c = 0;
+                            if (amax > 0.f && amax < INFINITY) {
+                                // c = 8 - ceil(log2 amax), read off the fp32 exponent and mantissa fields
+                                const uint32_t bits = __float_as_uint(amax);
+                                c = 8 - ((int)(bits >> 23) - 127 + ((bits & 0x7FFFFFu) != 0u ? 1 : 0));
+                                c = c < -100 ? -100 : (c > 100 ? 100 : c);
+                            }
+                            if (part == 0) {
+                                qsc[n] = __uint_as_float((uint32_t)(127 + c) << 23);
+                                qsc[NG + n] = __uint_as_float((uint32_t)(127 - c) << 23);
+                            }
+                        }
+                        named_bar_sync(SMX, NSM);
+                        // 8 columns at a time: hi codes to operand row n, lo codes to row NG + n
+                        for (int u = tid; u < NG * 72; u += NSM) {
+                            const int n = u / 72, w = u - 72 * n;
+                            const int ng = grp * NG + n;
+                            uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+                            if (ng < p.ncols)
+                                raw = __ldg(reinterpret_cast<const uint4 *>(p.q + ((int64_t)b * p.ncols + ng) * kDqk +
+                                                                            8 * w));
+                            const float sc = qsc[n];
+                            const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
+                            uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float a0 = __uint_as_float(wv[i] << 16) * sc;
+                                const float a1 = __uint_as_float(wv[i] & 0xFFFF0000u) * sc;
+                                const uint16_t h = f32x2_to_e4m3x2(a0, a1);
+                                const float2 hf = e4m3x2_to_f32x2(h);
+                                const uint16_t l = f32x2_to_e4m3x2(a0 - hf.x, a1 - hf.y);
+                                hi[i >> 1] |= (uint32_t)h << (16 * (i & 1));
+                                lo[i >> 1] |= (uint32_t)l << (16 * (i & 1));
+                            }
+                            uint32_t dh, dl;
+                            if (w < 64) {  // latent columns 8w..: chunk w / 16 (128 codes, 128B swizzle)
+                                const uint32_t base = C::OFF_Q + (uint32_t)(w >> 4) * C::Q_CHUNK;
+                                const uint32_t j16 = (uint32_t)(w & 15) >> 1, sub = (uint32_t)(w & 1) * 8u;
+                                dh = base + swz_off(n, j16, 128, 7) + sub;
+                                dl = base + swz_off(NG + n, j16, 128, 7) + sub;
+                            } else {  // rope columns: 64-byte rows, 64B swizzle
+                                const uint32_t w2 = (uint32_t)(w - 64), j16 = w2 >> 1, sub = (w2 & 1u) * 8u;
+                                dh = C::OFF_QR + swz_off(n, j16, C::R_ROW, 3) + sub;
+                                dl = C::OFF_QR + swz_off(NG + n, j16, C::R_ROW, 3) + sub;
+                            }
+                            *reinterpret_cast<uint2 *>(smem + dh) = make_uint2(hi[0], hi[1]);
+                            *reinterpret_cast<uint2 *>(smem + dl) = make_uint2(lo[0], lo[1]);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0 && !p.withhold_q) mbar_arrive(bar(BR::QFULL));
+                        ++qseg;
+                    }
+#pragma unroll
+                    for (int n = 0; n < NH; ++n) qv[n] = qsc[NG + 8 * half + n];
+                } else {
+#pragma unroll
+                    for (int n = 0; n < NH; ++n) qv[n] = 1.f;
+                }
+                for (int t = t0 + toff; t < t1 && !stop; t += C::TSTEP, ++k) {
+                    const bool first = (t == t0 + toff);
                     const int pb = k % C::PB;
                     ok = ok && spin_phase<false>(bar(BR::SFULL + (k & 1)), (k >> 1) & 1, wc, status);
                     tc_fence_after();
                     const int rg = t * kTileRows + row;
+                    // E4M3: this row's scale s (from the rope slot, which the warps then free); the row's scores
+                    // are s * (K codes . Q terms) * 2^-c_n, and the maximum tracks them plus log2 s
+                    float rsq[NH], lgs = 0.f, inv16 = 1.f;
+                    if constexpr (C::KV8) {
+                        const int rsl = k % C::NR;
+                        ok = ok && spin_phase<false>(bar(BR::RFULL + rsl), (k / C::NR) & 1, wc, status);
+                        float sig = *reinterpret_cast<const float *>(smem + C::OFF_R + rsl * C::R_SLOT + C::R_DATA +
+                                                                     4 * row);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(BR::REMPTY + rsl));
+                        sig = rg < L ? fmaxf(sig, 0x1p-100f) : 1.f;
+                        lgs = __log2f(sig);
+                        inv16 = 0.0625f / sig;  // 2^-4 / s: turns a stored p back into 2^(score - m)
+                        const float rsc = sig * p.scale_log2;
+#pragma unroll
+                        for (int n = 0; n < NH; ++n) rsq[n] = rsc * qv[n];
+                    } else {
+#pragma unroll
+                        for (int n = 0; n < NH; ++n) rsq[n] = p.scale_log2;
+                    }
                     // every row of the tile visible to every column: no per-column mask needed
                     const bool full_tile =
                         qlen_b == p.q_len && (t + 1) * kTileRows <= (p.causal ? L - qlen_b + 1 : L);
@@ -637,11 +829,22 @@ __global__ void __launch_bounds__(320, 1)
                     for (int ch = 0; ch < C::CH; ++ch) {
                         float(&x)[8] = xc[ch];
                         if constexpr (C::CH == 1) {
-                            tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * NG + 8 * half, x);
-                            tmem_wait_ld();
+                            tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * C::NS + 8 * half, x);
+                            if constexpr (C::KV8) {
+                                // scores against Q_hi and against Q_lo, added
+                                float xl[8];
+                                tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * C::NS + NG + 8 * half, xl);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int n = 0; n < 8; ++n) x[n] += xl[n];
+                            } else {
+                                tmem_wait_ld();
+                            }
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(bar(BR::SEMPTY + (k & 1)));
+                        }
+                        if constexpr (C::CH == 1 && !C::KV8) {
                             // Exchange of the partial scores with the peer CTA.  Slot xs is free for
                             // exchange e without a handshake: the peer overwrites it (exchange e + XS) only
                             // after receiving our exchange e + XS - 1, which we send after consuming e.
@@ -665,7 +868,18 @@ __global__ void __launch_bounds__(320, 1)
                                 x[4 * j + 3] += v.w;
                             }
                         }
-                        if (full_tile) {
+                        if constexpr (C::KV8) {
+                            if (full_tile) {
+#pragma unroll
+                                for (int n = 0; n < 8; ++n) x[n] = fmaf(x[n], rsq[8 * ch + n], lgs);
+                            } else {
+#pragma unroll
+                                for (int n = 0; n < 8; ++n) {
+                                    const int vis = __shfl_sync(0xffffffffu, vis_lane, 8 * ch + n);
+                                    x[n] = (rg < vis) ? fmaf(x[n], rsq[8 * ch + n], lgs) : -INFINITY;
+                                }
+                            }
+                        } else if (full_tile) {
 #pragma unroll
                             for (int n = 0; n < 8; ++n) x[n] *= p.scale_log2;
                         } else {
@@ -675,9 +889,9 @@ __global__ void __launch_bounds__(320, 1)
                                 x[n] = (rg < vis) ? x[n] * p.scale_log2 : -INFINITY;
                             }
                         }
-                        // running maximum: kept unless some row of the tile exceeds it by > 2^8
+                        // running maximum: kept unless some row of the tile exceeds it by > 2^THRESH
 #pragma unroll
-                        for (int n = 0; n < 8; ++n) need = need || (x[n] > m[8 * ch + n] + kRescaleThreshold);
+                        for (int n = 0; n < 8; ++n) need = need || (x[n] > m[8 * ch + n] + C::THRESH);
                     }
                     // ---- one vote per tile; the slow path takes the column maxima of all chunks
                     float alpha[C::CH][8];
@@ -716,10 +930,10 @@ __global__ void __launch_bounds__(320, 1)
                                 for (int u = 0; u < 4; ++u) {
                                     const int n = n4 + u, li = 8 * ch + n;
                                     if (first) {
-                                        m[li] = mt4[u] + kRescaleHeadroom;
-                                    } else if (mt4[u] > m[li] + kRescaleThreshold) {
-                                        alpha[ch][n] = fast_exp2(m[li] - (mt4[u] + kRescaleHeadroom));
-                                        m[li] = mt4[u] + kRescaleHeadroom;
+                                        m[li] = mt4[u] + C::HEADROOM;
+                                    } else if (mt4[u] > m[li] + C::THRESH) {
+                                        alpha[ch][n] = fast_exp2(m[li] - (mt4[u] + C::HEADROOM));
+                                        m[li] = mt4[u] + C::HEADROOM;
                                         rescale = true;
                                     }
                                 }
@@ -734,13 +948,38 @@ __global__ void __launch_bounds__(320, 1)
                         for (int n = 0; n < 8; ++n) {
                             const int li = 8 * ch + n;
                             const float mu = (m[li] == -INFINITY) ? 0.f : m[li];
-                            pv[n] = fast_exp2(xc[ch][n] - mu);
-                            lpart[li] = lpart[li] * alpha[ch][n] + pv[n];
+                            if constexpr (C::KV8) {
+                                // stored p = 2^(score + log2 s - m + 4); the sum takes 2^(score - m)
+                                pv[n] = fast_exp2(xc[ch][n] - (mu - kPScaleLog2_8));
+                                lpart[li] = fmaf(pv[n], inv16, lpart[li] * alpha[ch][n]);
+                            } else {
+                                pv[n] = fast_exp2(xc[ch][n] - mu);
+                                lpart[li] = lpart[li] * alpha[ch][n] + pv[n];
+                            }
                         }
                         // ---- P^T row chunk -> shared memory: bf16 hi into column 16ch+8half.., lo into NG + that
                         if (ch == 0)
                             ok = ok && spin_phase<false>(bar(BR::PEMPTY + pb), ((k / C::PB) & 1) ^ 1, wc, status);
-                        {
+                        if constexpr (C::KV8) {
+                            // P^T row chunk: E4M3 hi codes into columns 16ch+8half.., the residual's codes into NG + that
+                            uint32_t hi[2] = {0u, 0u}, lo[2] = {0u, 0u};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const uint16_t h = f32x2_to_e4m3x2(pv[2 * i], pv[2 * i + 1]);
+                                const float2 hf = e4m3x2_to_f32x2(h);
+                                const uint16_t l = f32x2_to_e4m3x2(pv[2 * i] - hf.x, pv[2 * i + 1] - hf.y);
+                                hi[i >> 1] |= (uint32_t)h << (16 * (i & 1));
+                                lo[i >> 1] |= (uint32_t)l << (16 * (i & 1));
+                            }
+                            uint8_t *pbuf = smem + C::OFF_P + pb * C::P_BUF;
+#pragma unroll
+                            for (int hl = 0; hl < 2; ++hl) {
+                                const int col0 = hl * NG + 16 * ch + 8 * half;  // first P^T column (= byte) of these 8
+                                *reinterpret_cast<uint2 *>(pbuf + swz_off(row, col0 / 16, C::P_PITCH, C::P_SWZ_MASK) +
+                                                           (col0 % 16)) =
+                                    hl == 0 ? make_uint2(hi[0], hi[1]) : make_uint2(lo[0], lo[1]);
+                            }
+                        } else {
                             uint32_t hi[4], lo[4];
 #pragma unroll
                             for (int n = 0; n < 8; n += 2) {
@@ -773,7 +1012,7 @@ __global__ void __launch_bounds__(320, 1)
                             }
                             rescale_any = true;
 #pragma unroll
-                            for (int i = 0; i < C::PAIRS; ++i) {
+                            for (int i = 0; i < C::MB; ++i) {
 #pragma unroll
                                 for (int hl = 0; hl < 2; ++hl) {
                                     float v[8];
@@ -811,7 +1050,8 @@ __global__ void __launch_bounds__(320, 1)
                 if (stop) break;
                 // ---------------------------------------------------- epilogue: step 4 for this CTA's 256 columns
                 const int kl = k - 1;
-                ok = ok && spin_phase<false>(bar(BR::PEMPTY + (kl % C::PB)), (kl / C::PB) & 1, wc, status);
+                if (has_tiles)  // the last step 3 of this segment has completed
+                    ok = ok && spin_phase<false>(bar(BR::PEMPTY + (kl % C::PB)), (kl / C::PB) & 1, wc, status);
                 tc_fence_after();
 #pragma unroll
                 for (int ch = 0; ch < C::CH; ++ch) {
@@ -827,35 +1067,17 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 const int nsplit = seg_nsplit;
                 const int slot = seg_slot;
-#pragma unroll
-                for (int ch = 0; ch < C::CH; ++ch) {
-                    float inv_l[8], lse_n[8];
-#pragma unroll
-                    for (int n = 0; n < 8; ++n) {
-                        const int cn = 16 * ch + 8 * half + n, li = 8 * ch + n;
-                        const float l = redl[cn] + redl[NG + cn] + redl[2 * NG + cn] + redl[3 * NG + cn];
-                        const bool empty = !(l > 0.f) || m[li] == -INFINITY;
-                        inv_l[n] = empty ? 0.f : 1.f / l;
-                        lse_n[n] = empty ? -INFINITY : (m[li] + __log2f(l)) * 0.69314718055994531f;
-                    }
-#pragma unroll
-                    for (int i = 0; i < C::PAIRS; ++i) {
-                        float hi[8], lo[8];
-                        tmem_ld8(tmem + lane_addr + C::O_COL + i * C::NP + 16 * ch + 8 * half, hi);
-                        tmem_ld8(tmem + lane_addr + C::O_COL + i * C::NP + NG + 16 * ch + 8 * half, lo);
-                        tmem_wait_ld();
-                        const int d = 256 * (int)rank + 128 * i + row;
-#pragma unroll
-                        for (int n = 0; n < 8; ++n) {
-                            const int ng = grp * NG + 16 * ch + 8 * half + n;
-                            if (ng >= p.ncols) continue;
-                            const float val = (hi[n] + lo[n]) * inv_l[n];
-                            if (nsplit == 1)
-                                p.o[((int64_t)b * p.ncols + ng) * kDv + d] = __float2bfloat16_rn(val);
-                            else
-                                p.opart[((int64_t)slot * p.ncols + ng) * kDv + d] = val;
-                        }
-                    }
+                // this CTA's result for latent row d = 256 rank + 128 i + row of column 16 ch + 8 half + n
+                auto store_o = [&](int ch, int i, int n, float val) {
+                    const int d = 256 * (int)rank + 128 * i + row;
+                    const int ng = grp * NG + 16 * ch + 8 * half + n;
+                    if (ng >= p.ncols) return;
+                    if (nsplit == 1)
+                        p.o[((int64_t)b * p.ncols + ng) * kDv + d] = __float2bfloat16_rn(val);
+                    else
+                        p.opart[((int64_t)slot * p.ncols + ng) * kDv + d] = val;
+                };
+                auto store_lse = [&](int ch, const float (&lse_n)[8]) {
                     if (quad == 0 && lane < 8) {
                         const int ng = grp * NG + 16 * ch + 8 * half + lane;
                         float my = lse_n[0];
@@ -870,6 +1092,126 @@ __global__ void __launch_bounds__(320, 1)
                             }
                         }
                     }
+                };
+                if constexpr (C::KV8) {
+                    // ---- merge of the two CTAs' partials of this segment (disjoint tiles, all 512 latent rows
+                    //      each): send the peer the two M-tiles it writes and this CTA's (m, l) of these columns,
+                    //      receive the same, and combine by the log-sum-exp rule.
+                    float ms[8], ls[8], ov[4][8];
+#pragma unroll
+                    for (int n = 0; n < 8; ++n) {
+                        const int cn = 8 * half + n;
+                        ls[n] = redl[cn] + redl[NG + cn] + redl[2 * NG + cn] + redl[3 * NG + cn];
+                        ms[n] = has_tiles ? m[n] : -INFINITY;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float hi[8], lo[8];
+                        if (has_tiles) {
+                            tmem_ld8(tmem + lane_addr + C::O_COL + i * C::NP + 8 * half, hi);
+                            tmem_ld8(tmem + lane_addr + C::O_COL + i * C::NP + NG + 8 * half, lo);
+                            tmem_wait_ld();
+                        }
+#pragma unroll
+                        for (int n = 0; n < 8; ++n) ov[i][n] = has_tiles ? hi[n] + lo[n] : 0.f;
+                    }
+                    tc_fence_before();
+                    // M-tiles 2 rank, 2 rank + 1 stay here, the other two go to the peer (selects, so that
+                    // nothing is indexed by the rank at run time)
+                    float own[2][8], oth[2][8];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+#pragma unroll
+                        for (int n = 0; n < 8; ++n) {
+                            own[j][n] = rank == 0 ? ov[j][n] : ov[2 + j][n];
+                            oth[j][n] = rank == 0 ? ov[2 + j][n] : ov[j][n];
+                        }
+                    const uint32_t x_peer = map_to_rank(sbase + C::OFF_X, peer);
+                    const uint32_t xrow = (uint32_t)row * 64u + (uint32_t)half * 32u;
+                    const uint32_t xml = 2u * 8192u + (uint32_t)sw * 64u;
+                    ok = ok && spin_phase<true>(bar(BR::XFREE + sw), (mseg & 1) ^ 1, wc, status);
+                    if (ok) {
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const float *v = oth[j];
+                            st_async_v4(x_peer + 8192u * j + xrow, __float_as_uint(v[0]), __float_as_uint(v[1]),
+                                        __float_as_uint(v[2]), __float_as_uint(v[3]), xfull_remote);
+                            st_async_v4(x_peer + 8192u * j + xrow + 16u, __float_as_uint(v[4]), __float_as_uint(v[5]),
+                                        __float_as_uint(v[6]), __float_as_uint(v[7]), xfull_remote);
+                        }
+                        if (lane == 0) {
+                            st_async_v4(x_peer + xml, __float_as_uint(ms[0]), __float_as_uint(ms[1]),
+                                        __float_as_uint(ms[2]), __float_as_uint(ms[3]), xfull_remote);
+                            st_async_v4(x_peer + xml + 16u, __float_as_uint(ms[4]), __float_as_uint(ms[5]),
+                                        __float_as_uint(ms[6]), __float_as_uint(ms[7]), xfull_remote);
+                            st_async_v4(x_peer + xml + 32u, __float_as_uint(ls[0]), __float_as_uint(ls[1]),
+                                        __float_as_uint(ls[2]), __float_as_uint(ls[3]), xfull_remote);
+                            st_async_v4(x_peer + xml + 48u, __float_as_uint(ls[4]), __float_as_uint(ls[5]),
+                                        __float_as_uint(ls[6]), __float_as_uint(ls[7]), xfull_remote);
+                        }
+                    }
+                    if (lane == 0) mbar_arrive_expect_tx(bar(BR::XFULL + sw), 32 * 64 + 64);
+                    ok = ok && spin_phase<true>(bar(BR::XFULL + sw), mseg & 1, wc, status);
+                    ++mseg;
+                    float op[2][8], mp[8], lp[8];
+                    {
+                        const float *xs = reinterpret_cast<const float *>(smem + C::OFF_X);
+#pragma unroll
+                        for (int j = 0; j < 2; ++j)
+#pragma unroll
+                            for (int n = 0; n < 8; ++n) op[j][n] = xs[(8192u * j + xrow) / 4 + n];
+#pragma unroll
+                        for (int n = 0; n < 8; ++n) {
+                            mp[n] = xs[xml / 4 + n];
+                            lp[n] = xs[xml / 4 + 8 + n];
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(xfree_remote);
+                    if (!named_bar_and(SMX, NSM, ok)) {
+                        stop = true;
+                        break;
+                    }
+                    float lse_n[8];
+#pragma unroll
+                    for (int n = 0; n < 8; ++n) {
+                        const float mm = fmaxf(ms[n], mp[n]);
+                        const float as = ms[n] == -INFINITY ? 0.f : fast_exp2(ms[n] - mm);
+                        const float ap = mp[n] == -INFINITY ? 0.f : fast_exp2(mp[n] - mm);
+                        const float l = ls[n] * as + lp[n] * ap;
+                        const bool empty = !(l > 0.f) || mm == -INFINITY;
+                        // the stored p carried a factor 2^4
+                        const float inv = empty ? 0.f : 0.0625f / l;
+                        lse_n[n] = empty ? -INFINITY : (mm + __log2f(l)) * 0.69314718055994531f;
+#pragma unroll
+                        for (int j = 0; j < 2; ++j)
+                            store_o(0, j, n, (own[j][n] * as + op[j][n] * ap) * inv);
+                    }
+                    store_lse(0, lse_n);
+                } else {
+#pragma unroll
+                for (int ch = 0; ch < C::CH; ++ch) {
+                    float inv_l[8], lse_n[8];
+
+#pragma unroll
+                    for (int n = 0; n < 8; ++n) {
+                        const int cn = 16 * ch + 8 * half + n, li = 8 * ch + n;
+                        const float l = redl[cn] + redl[NG + cn] + redl[2 * NG + cn] + redl[3 * NG + cn];
+                        const bool empty = !(l > 0.f) || m[li] == -INFINITY;
+                        inv_l[n] = empty ? 0.f : 1.f / l;
+                        lse_n[n] = empty ? -INFINITY : (m[li] + __log2f(l)) * 0.69314718055994531f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < C::MB; ++i) {
+                        float hi[8], lo[8];
+                        tmem_ld8(tmem + lane_addr + C::O_COL + i * C::NP + 16 * ch + 8 * half, hi);
+                        tmem_ld8(tmem + lane_addr + C::O_COL + i * C::NP + NG + 16 * ch + 8 * half, lo);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int n = 0; n < 8; ++n) store_o(ch, i, n, (hi[n] + lo[n]) * inv_l[n]);
+                    }
+                    store_lse(ch, lse_n);
+                }
                 }
                 if (nsplit >= 2 && p.fuse_merge) {
                     // Split-KV merge in the kernel: the last CTA (of this rank) to finish a split of

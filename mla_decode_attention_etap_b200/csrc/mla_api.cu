@@ -46,21 +46,26 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor map over a [rows, 576] row-major matrix; box = box_cols columns x box_rows rows,
-// 128B swizzle for 64-column boxes, 64B swizzle for the 32-column rope boxes.
-int encode_rows_576(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows, uint32_t box_cols = 64) {
+// 2-D tensor map over a [rows, 576] row-major matrix of bf16 (elem_bytes 2) or E4M3 codes
+// (elem_bytes 1); box = box_cols columns x box_rows rows, swizzled by the box's row width
+// (128 bytes: 128B swizzle, 64: 64B, 32: 32B), as the MMA operand descriptors expect.
+int encode_rows_576(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows, uint32_t box_cols = 64,
+                    uint32_t elem_bytes = 2) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) {
         g_last_cuda_error = "cuTensorMapEncodeTiled unavailable";
         return MLA_ERR_CUDA;
     }
     cuuint64_t dims[2] = {(cuuint64_t)mla::kDqk, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)mla::kDqk * 2};
+    cuuint64_t strides[1] = {(cuuint64_t)mla::kDqk * elem_bytes};
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+    const uint32_t row_bytes = box_cols * elem_bytes;
+    CUresult r = enc(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     row_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                     : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                       : CU_TENSOR_MAP_SWIZZLE_32B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         g_last_cuda_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string((int)r);
@@ -92,6 +97,9 @@ int ensure_smem_attr() {
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)mla::PairCfg32::SMEM_ALLOC);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg16E4>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::PairCfg16E4::SMEM_ALLOC);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         done[dev] = true;
     }
@@ -238,12 +246,20 @@ int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const 
                                  softmax_scale, causal, o, lse, workspace, workspace_bytes, num_sms, flags, stream);
 }
 
-int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *seqlens, const int32_t *q_lens,
-                          const int32_t *block_table, int batch, int q_len, int num_heads, int64_t kv_rows,
-                          int max_blocks, float softmax_scale, int causal, void *o, float *lse, void *workspace,
-                          size_t workspace_bytes, int num_sms, unsigned flags, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Validation, tensor maps and launch shared by the bf16 and E4M3 cache entry points
+// (kv_scale != NULL selects the E4M3 cache).
+int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const int32_t *seqlens,
+                    const int32_t *q_lens, const int32_t *block_table, int batch, int q_len, int num_heads,
+                    int64_t kv_rows, int max_blocks, float softmax_scale, int causal, void *o, float *lse,
+                    void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream) {
+    const bool fp8 = kv_scale != nullptr;
     int st = check_shape(batch, q_len, num_heads, num_sms);
     if (st != MLA_OK) return st;
+    if (fp8 && q_len * num_heads > 16) return MLA_ERR_UNSUPPORTED;
     if (!q || !kv || !seqlens || !o || !lse || !workspace) return MLA_ERR_INVALID_ARG;
     if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
@@ -258,7 +274,7 @@ int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *seqlens,
         if ((int64_t)batch * kv_rows > INT32_MAX) return MLA_ERR_UNSUPPORTED;
     }
     if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(o, 16) || !aligned(lse, 4) || !aligned(seqlens, 4) ||
-        !aligned(workspace, 256) || !aligned(q_lens, 4))
+        !aligned(workspace, 256) || !aligned(q_lens, 4) || !aligned(kv_scale, 4))
         return MLA_ERR_ALIGNMENT;
     const mla::WsLayout lay = mla::ws_layout(batch, q_len, num_heads, num_sms);
     if (workspace_bytes < lay.total) return MLA_ERR_WORKSPACE;
@@ -269,17 +285,29 @@ int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *seqlens,
     CUtensorMap tm_q, tm_kv, tm_qr, tm_kvr;
     const int ng = mla::group_cols(ncols);
     const uint64_t kv_total_rows = paged ? (uint64_t)kv_rows : (uint64_t)batch * kv_rows;
-    st = encode_rows_576(&tm_q, q, (uint64_t)batch * ncols, (uint32_t)ng);
-    if (st != MLA_OK) return st;
-    st = encode_rows_576(&tm_kv, kv, kv_total_rows, 64);
-    if (st != MLA_OK) return st;
-    st = encode_rows_576(&tm_qr, q, (uint64_t)batch * ncols, (uint32_t)ng, 32);
-    if (st != MLA_OK) return st;
-    st = encode_rows_576(&tm_kvr, kv, kv_total_rows, 64, 32);
-    if (st != MLA_OK) return st;
+    if (fp8) {
+        // the E4M3 kernel quantises Q itself (no Q maps): 128-code boxes of the latent part, 64-code rope boxes
+        st = encode_rows_576(&tm_kv, kv, kv_total_rows, 64, 128, 1);
+        if (st != MLA_OK) return st;
+        st = encode_rows_576(&tm_kvr, kv, kv_total_rows, 64, 64, 1);
+        if (st != MLA_OK) return st;
+        tm_q = tm_kv;
+        tm_qr = tm_kvr;
+    } else {
+        st = encode_rows_576(&tm_q, q, (uint64_t)batch * ncols, (uint32_t)ng);
+        if (st != MLA_OK) return st;
+        st = encode_rows_576(&tm_kv, kv, kv_total_rows, 64);
+        if (st != MLA_OK) return st;
+        st = encode_rows_576(&tm_qr, q, (uint64_t)batch * ncols, (uint32_t)ng, 32);
+        if (st != MLA_OK) return st;
+        st = encode_rows_576(&tm_kvr, kv, kv_total_rows, 64, 32);
+        if (st != MLA_OK) return st;
+    }
 
     char *ws = reinterpret_cast<char *>(workspace);
     mla::DecodeParams p{};
+    p.q = reinterpret_cast<const __nv_bfloat16 *>(q);
+    p.kv_scale = kv_scale;
     p.seqlens = seqlens;
     p.q_lens = q_lens;
     p.block_table = block_table;
@@ -307,18 +335,44 @@ int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *seqlens,
     p.counters = reinterpret_cast<int32_t *>(ws + lay.counters);
     p.slots = lay.slots;
     // splits of a sequence are at most the work units (CTA pairs per column group)
-    const int max_splits = ng == 16 ? mla::PairCfg16::MERGE_MAX_SPLITS : mla::PairCfg32::MERGE_MAX_SPLITS;
+    const int max_splits = fp8        ? mla::PairCfg16E4::MERGE_MAX_SPLITS
+                           : ng == 16 ? mla::PairCfg16::MERGE_MAX_SPLITS
+                                      : mla::PairCfg32::MERGE_MAX_SPLITS;
     const bool separate_combine = !(flags & MLA_FLAG_SKIP_COMBINE) && lay.ctas > max_splits;
     p.fuse_merge = ((flags & MLA_FLAG_SKIP_COMBINE) || separate_combine) ? 0 : 1;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = ng == 16 ? launch_pair<mla::PairCfg16>(tm_q, tm_kv, tm_qr, tm_kvr, p, lay.ctas * lay.groups, s)
-                             : launch_pair<mla::PairCfg32>(tm_q, tm_kv, tm_qr, tm_kvr, p, lay.ctas * lay.groups, s);
+    const int clusters = lay.ctas * lay.groups;
+    cudaError_t e = fp8        ? launch_pair<mla::PairCfg16E4>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s)
+                    : ng == 16 ? launch_pair<mla::PairCfg16>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s)
+                               : launch_pair<mla::PairCfg32>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s);
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
     if (separate_combine) return mla_combine(workspace, batch, q_len, num_heads, num_sms, o, lse, stream);
     return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *seqlens, const int32_t *q_lens,
+                          const int32_t *block_table, int batch, int q_len, int num_heads, int64_t kv_rows,
+                          int max_blocks, float softmax_scale, int causal, void *o, float *lse, void *workspace,
+                          size_t workspace_bytes, int num_sms, unsigned flags, void *stream) {
+    return decode_fwd_impl(q, kv, nullptr, seqlens, q_lens, block_table, batch, q_len, num_heads, kv_rows, max_blocks,
+                           softmax_scale, causal, o, lse, workspace, workspace_bytes, num_sms, flags, stream);
+}
+
+int mla_decode_fwd_fp8(const void *q, const void *kv8, const float *kv_scale, const int32_t *seqlens,
+                       const int32_t *q_lens, const int32_t *block_table, int batch, int q_len, int num_heads,
+                       int64_t kv_rows, int max_blocks, float softmax_scale, int causal, void *o, float *lse,
+                       void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream) {
+    if (!kv_scale) return MLA_ERR_INVALID_ARG;
+    return decode_fwd_impl(q, kv8, kv_scale, seqlens, q_lens, block_table, batch, q_len, num_heads, kv_rows,
+                           max_blocks, softmax_scale, causal, o, lse, workspace, workspace_bytes, num_sms, flags,
+                           stream);
 }
 
 int mla_stream_probe(const void *kv, int64_t rows, int units, int32_t *err, void *stream) {

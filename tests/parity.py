@@ -31,7 +31,11 @@ def run_cuda(w: Workload, n_sms=None, flags=0, poison=True, decoder=None):
                      dtype=torch.float32, device=dev)
     dec.plan(sl)
     ql = w.q_lens.to(dev) if w.q_lens is not None else None
-    dec.fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o=o, lse=lse, flags=flags, q_lens=ql)
+    if w.fp8:
+        dec.fwd_fp8(q, w.kv8.to(dev), w.kv_scale.to(dev), sl, bt, w.softmax_scale, w.causal, o=o, lse=lse,
+                    flags=flags, q_lens=ql)
+    else:
+        dec.fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o=o, lse=lse, flags=flags, q_lens=ql)
     torch.cuda.synchronize()
     status = dec.status()
     return o.float().cpu().numpy(), lse.cpu().numpy(), status, dec
@@ -39,6 +43,8 @@ def run_cuda(w: Workload, n_sms=None, flags=0, poison=True, decoder=None):
 
 def run_oracle(w: Workload, batch_index=None):
     """fp64 oracle on all sequences, or on the listed ones (each resolved to a contiguous copy)."""
+    if w.fp8:
+        return _run_oracle_fp8(w, batch_index)
     if batch_index is None:
         q = bf16_bits(w.q)
         kv = bf16_bits(w.kv)
@@ -53,6 +59,34 @@ def run_oracle(w: Workload, batch_index=None):
         q = bf16_bits(w.q[b:b + 1].cpu())
         ql = None if w.q_lens is None else w.q_lens[b:b + 1].numpy()
         o, lse = om.mla_decode(q, kv, np.array([L], np.int32), None, w.softmax_scale, w.causal, q_lens=ql)
+        outs_o.append(o[0])
+        outs_l.append(lse[0])
+    return np.stack(outs_o), np.stack(outs_l)
+
+
+def _seq_rows(w: Workload, t: torch.Tensor, b: int) -> torch.Tensor:
+    """Logical rows [L_b, ...] of a per-row cache tensor (codes or scales) of sequence b."""
+    L = int(w.seqlens[b])
+    if w.block_table is None:
+        return t[b, :L]
+    nb = (L + 63) // 64
+    return t[w.block_table[b, :nb].long()].reshape(nb * 64, *t.shape[2:])[:L]
+
+
+def _run_oracle_fp8(w: Workload, batch_index):
+    if batch_index is None:
+        bt = None if w.block_table is None else w.block_table.numpy()
+        ql = None if w.q_lens is None else w.q_lens.numpy()
+        return om.mla_decode_fp8(bf16_bits(w.q), w.kv8.numpy(), w.kv_scale.numpy(), w.seqlens.numpy(), bt,
+                                 w.softmax_scale, w.causal, q_lens=ql)
+    outs_o, outs_l = [], []
+    for b in batch_index:
+        L = int(w.seqlens[b])
+        codes = _seq_rows(w, w.kv8, b).numpy().reshape(1, L, 576) if L > 0 else np.zeros((1, 1, 576), np.uint8)
+        sc = _seq_rows(w, w.kv_scale, b).numpy().reshape(1, L) if L > 0 else np.ones((1, 1), np.float32)
+        ql = None if w.q_lens is None else w.q_lens[b:b + 1].numpy()
+        o, lse = om.mla_decode_fp8(bf16_bits(w.q[b:b + 1].cpu()), codes, sc, np.array([L], np.int32), None,
+                                   w.softmax_scale, w.causal, q_lens=ql)
         outs_o.append(o[0])
         outs_l.append(lse[0])
     return np.stack(outs_o), np.stack(outs_l)

@@ -1,0 +1,173 @@
+"""GPU parity of the FP8-cache decode (E4M3 codes + one fp32 scale per cache row) against the
+fp64 oracle on the same codes and scales, through the C ABI (``mla_decode_fwd_fp8``).
+
+Same bar as the bf16 path: RMSE(O) <= 2e-3 RMS(O_ref), max|O - O_ref| <= 1e-2 max|O_ref|,
+|LSE - LSE_ref| <= 1e-3.  Cache rows past L_b hold NaN codes (0x7F) and NaN scales."""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from mla_decode_attention_etap_b200 import MlaDecoder, MlaError
+from mla_decode_attention_etap_b200 import workloads as W
+from tests.parity import assert_parity, run_cuda, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+NAN_CODE = 0x7F
+
+
+def _poison(w):
+    """NaN codes and NaN scales in every cache row that no sequence reads."""
+    if w.block_table is None:
+        for b in range(w.batch):
+            L = int(w.seqlens[b])
+            w.kv8[b, L:] = NAN_CODE
+            w.kv_scale[b, L:] = float("nan")
+    else:
+        used = set()
+        for b in range(w.batch):
+            L = int(w.seqlens[b])
+            nb = (L + 63) // 64
+            for i in range(nb):
+                blk = int(w.block_table[b, i])
+                used.add(blk)
+                n = L - 64 * i
+                if n < 64:
+                    w.kv8[blk, n:] = NAN_CODE
+                    w.kv_scale[blk, n:] = float("nan")
+        for blk in range(w.kv8.shape[0]):
+            if blk not in used:
+                w.kv8[blk] = NAN_CODE
+                w.kv_scale[blk] = float("nan")
+    return w
+
+
+def fp8(*args, **kw):
+    return W.make_workload(*args, kv_dtype="e4m3", **kw)
+
+
+@pytest.mark.parametrize("L", [1, 2, 63, 64, 65, 127, 128, 129, 640, 1000, 4097])
+def test_edge_lengths(L):
+    w = _poison(fp8(1, 16, [L], seed=100 + L, l_max=L + 200))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"fp8 L={L}")
+
+
+def test_b1_h16_l1024():
+    w = fp8(1, 16, [1024], seed=0)
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what="fp8 B=1 L=1024")
+
+
+def test_mixed_lengths_with_empty_sequences():
+    lens = [0, 1, 129, 700, 64, 2000, 3, 0]
+    w = _poison(fp8(len(lens), 16, lens, seed=101))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert np.all(o[0] == 0) and np.all(np.isneginf(lse[0])) and np.all(np.isneginf(lse[7]))
+    assert_parity(o, lse, *run_oracle(w), what="fp8 mixed")
+
+
+@pytest.mark.parametrize("n_sms", [1, 3, 16, 148, 300, 1024])
+def test_split_counts(n_sms):
+    w = fp8(3, 16, [3000, 257, 1536], seed=102)
+    o, lse, st, _ = run_cuda(w, n_sms=n_sms)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"fp8 n_sms={n_sms}")
+
+
+def test_paged_with_poisoned_pool():
+    lens = [1, 4000, 64, 65, 900, 0, 2500]
+    w = _poison(fp8(len(lens), 16, lens, paged=True, seed=103, extra_blocks=9))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what="fp8 paged")
+
+
+def test_spiky_rows_and_causal_multi_token():
+    # rows scaled x8 (their E4M3 scale grows, the codes do not), 2 causal tokens x 8 heads
+    w = _poison(fp8(2, 8, [3000, 129], q_len=2, causal=True, seed=104, spike_frac=0.05, l_max=3100))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what="fp8 causal q2")
+
+
+def test_ragged_query_counts():
+    w = _poison(fp8(4, 4, [500, 90, 1300, 7], q_len=4, causal=True, seed=105, q_lens=[4, 1, 0, 3],
+                    l_max=1400))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert np.all(o[2] == 0) and np.all(np.isneginf(lse[2]))
+    assert_parity(o, lse, *run_oracle(w), what="fp8 ragged")
+
+
+@pytest.mark.parametrize("h", [1, 5, 12])
+def test_fewer_heads_than_columns(h):
+    w = fp8(2, h, [777, 2049], seed=106 + h)
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"fp8 h={h}")
+
+
+def test_query_columns_of_very_different_magnitude():
+    """Each query column gets its own power-of-two factor before its E4M3 split."""
+    w = fp8(2, 16, [1500, 300], seed=107)
+    f = torch.tensor([2.0 ** e for e in (-12, -6, -1, 0, 3, 7, 9, 11, 0, -3, 5, -9, 2, 1, -2, 4)])
+    w.q = (w.q.float() * f[None, None, :, None]).to(torch.bfloat16)
+    w.softmax_scale = 1.0 / 24.0 / 64.0  # keeps the large columns' scores finite and not one-hot
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what="fp8 column magnitudes")
+
+
+@pytest.mark.parametrize("scale_factor", [2.0 ** -40, 16.0])
+def test_row_scales_far_from_one(scale_factor):
+    # (much larger factors make |LSE| so large that an fp32 LSE cannot hold the 1e-3 bound)
+    w = fp8(2, 16, [1000, 333], seed=108)
+    w.kv_scale *= scale_factor
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"fp8 scales x {scale_factor}")
+
+
+def test_skip_combine_then_combine_matches():
+    from mla_decode_attention_etap_b200 import FLAG_SKIP_COMBINE, mla_combine
+    w = fp8(3, 16, [5000, 700, 2100], seed=109)
+    dev = torch.device("cuda")
+    o1, l1, st, dec = run_cuda(w)
+    assert st == 0
+    o = torch.zeros(w.batch, 1, 16, 512, dtype=torch.bfloat16, device=dev)
+    lse = torch.zeros(w.batch, 1, 16, dtype=torch.float32, device=dev)
+    sl = w.seqlens.to(dev)
+    dec.plan(sl)
+    dec.fwd_fp8(w.q.to(dev), w.kv8.to(dev), w.kv_scale.to(dev), sl, None, w.softmax_scale, False, o=o, lse=lse,
+                flags=FLAG_SKIP_COMBINE)
+    mla_combine(dec.workspace, w.batch, 1, 16, dec.n_sms, o, lse)
+    torch.cuda.synchronize()
+    assert np.array_equal(o.float().cpu().numpy(), o1) and np.array_equal(lse.cpu().numpy(), l1)
+
+
+def test_full_size_64k_sampled_sequences():
+    """B=16, h=16, 65536 rows in the launch configuration bench.py times: sequences 0, 7, 15 vs the oracle."""
+    w = W.workload_b16_h16_fp8(65536, seed=0)
+    o, lse, st, _ = run_cuda(w, poison=False)
+    assert st == 0
+    idx = [0, 7, 15]
+    o_ref, lse_ref = run_oracle(w, batch_index=idx)
+    assert_parity(o[idx], lse[idx], o_ref, lse_ref, what="fp8 64K sampled")
+
+
+def test_unsupported_column_count_is_rejected():
+    w = fp8(1, 32, [100], seed=110)
+    dev = torch.device("cuda")
+    dec = MlaDecoder(1, 1, 32, device=dev)
+    sl = w.seqlens.to(dev)
+    dec.plan(sl)
+    with pytest.raises(MlaError) as ei:
+        dec.fwd_fp8(w.q.to(dev), w.kv8.to(dev), w.kv_scale.to(dev), sl)
+    assert ei.value.code == -2
