@@ -47,6 +47,7 @@ KERNEL_SOURCES = ["mla_decode_attention_etap_b200/csrc/etap_pair_kernel.cuh",
                   "mla_decode_attention_etap_b200/csrc/plan_core.h",
                   "mla_decode_attention_etap_b200/csrc/merge.cuh"]
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "etap_pair_kernel_ncu.md")
+PROFILE_SUMMARIES = [PROFILE_SUMMARY, os.path.join(ROOT, "profiles", "etap_pair_kernel_e4m3_ncu.md")]
 
 WORKLOADS = {
     "b16_h16_64k": dict(batch=16, heads=16, seqlen=65536),
@@ -156,16 +157,19 @@ def kernel_source_hash(read=None) -> str:
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if taken on the current kernel source."""
-    try:
-        text = open(PROFILE_SUMMARY).read()
-    except OSError:
-        return None
-    src = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
-    if not src or src.group(1) != kernel_source_hash():
-        return None
-    m = re.search(rf"traffic_bytes_per_launch\[{re.escape(workload)}\]:\s*([0-9.eE+]+)", text)
-    return float(m.group(1)) if m else None
+    """DRAM bytes per decode launch from the committed ncu summaries, if taken on the current kernel source."""
+    for path in PROFILE_SUMMARIES:
+        try:
+            text = open(path).read()
+        except OSError:
+            continue
+        src = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+        if not src or src.group(1) != kernel_source_hash():
+            continue
+        m = re.search(rf"traffic_bytes_per_launch\[{re.escape(workload)}\]:\s*([0-9.eE+]+)", text)
+        if m:
+            return float(m.group(1))
+    return None
 
 
 # ---------------------------------------------------------------- clocks
