@@ -59,6 +59,7 @@ WORKLOADS = {
     "b32_h128_paged": dict(kind="b32_h128"),
     "b16_h16_q4_causal": dict(kind="q4_causal"),
     "b16_h16_ragged_q4_causal": dict(kind="ragged_q4_causal"),
+    "b16_h16_append_q16": dict(kind="append_q16"),
     # FP8 latent cache (E4M3 codes + one fp32 scale per row): 580 bytes per cached token
     "b16_h16_64k_fp8": dict(batch=16, heads=16, seqlen=65536, fp8=True),
     "b16_h16_16k_fp8": dict(batch=16, heads=16, seqlen=16384, fp8=True),
@@ -113,6 +114,9 @@ def make_workload(name: str, rank: int, device):
     if kind == "ragged_q4_causal":
         return (W.workload_b16_h16_ragged_q4_causal(seed=seed, device=device),
                 "mla_decode_b16_h16_ragged_q1to4_causal_L32768_spikes5pct_x8")
+    if kind == "append_q16":
+        return (W.workload_b16_h16_append_q16(seed=seed, device=device),
+                "mla_decode_b16_h16_append_q16_causal_L32768")
     if kind == "b64_paged_fp8":
         return (W.workload_b64_h16_paged_fp8(seed=seed, device=device),
                 "mla_decode_b64_h16_q1_Lunif1to65536_paged64_e4m3cache")

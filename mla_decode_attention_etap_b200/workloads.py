@@ -220,6 +220,12 @@ def workload_b16_h16_ragged_q4_causal(seed: int = 0, device="cpu", seqlen: int =
                          spike_frac=0.05, spike_scale=8.0, q_lens=q_lens)
 
 
+def workload_b16_h16_append_q16(seed: int = 0, device="cpu", seqlen: int = 32768, batch: int = 16) -> Workload:
+    """Append attention: B=16, 16 heads, 16 new causal tokens at the end of a 32768-row cache
+    (256 query columns per sequence)."""
+    return make_workload(batch, 16, [seqlen] * batch, q_len=16, causal=True, seed=seed, device=device)
+
+
 def workload_b16_h16_fp8(seqlen: int, seed: int = 0, device="cpu") -> Workload:
     """B=16, 16 heads, one query token, equal contiguous lengths, FP8 (E4M3 + row scale) cache."""
     return make_workload(16, 16, [seqlen] * 16, seed=seed, device=device, kv_dtype="e4m3")

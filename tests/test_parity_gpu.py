@@ -351,3 +351,32 @@ def test_cuda_graph_replay_matches_eager():
         torch.cuda.synchronize()
         assert torch.equal(o, o_eager) and torch.equal(lse, l_eager)
     assert dec.status() == 0
+
+
+@pytest.mark.parametrize("q_len,lens", [(8, [700, 8]), (16, [1500, 40, 17]), (32, [2100, 333]), (64, [1000, 64, 65])])
+def test_append_causal_moderate_q_len(q_len, lens):
+    """Append attention: q_len = 8..64 new tokens per sequence, causal, 16 heads (N = 128..1024 query
+    columns in groups of 32); includes caches barely longer than the appended tokens."""
+    w = _poison_padding(W.make_workload(len(lens), 16, lens, q_len=q_len, causal=True, seed=70 + q_len,
+                                        l_max=max(lens) + 50, spike_frac=0.02))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"append q_len={q_len}")
+
+
+def test_append_ragged_paged():
+    """Append with a different number of new tokens per sequence (0..16) on a paged cache."""
+    lens = [900, 16, 1300, 5]
+    q_lens = [16, 16, 3, 0]
+    w = _poison_padding(W.make_workload(len(lens), 16, lens, q_len=16, causal=True, paged=True, seed=80,
+                                        q_lens=q_lens))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    for b, qb in enumerate(q_lens):
+        assert np.all(o[b, qb:] == 0) and np.all(np.isneginf(lse[b, qb:]))
+    assert_parity(o, lse, *run_oracle(w), what="append ragged paged")
+
+
+def test_full_b16_h16_append_q16_sampled():
+    w = W.workload_b16_h16_append_q16(seed=0, device="cuda")
+    _full(w, [0, 9])
