@@ -553,6 +553,39 @@ def run_ours(args):
     return 0
 
 
+def run_ablation(args):
+    """Transposed vs untransposed contraction cost per 128-row KV tile (the pages' padding argument):
+    tensor-core instructions only, every SM, h in {16, 32, 64, 128}; one JSON line."""
+    import torch
+    import mla_decode_attention_etap_b200 as mla
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    ctas = torch.cuda.get_device_properties(dev).multi_processor_count
+    tiles = 64
+    cycles = torch.zeros(ctas, dtype=torch.int64, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    rows = []
+    for heads in (16, 32, 64, 128):
+        entry = {"heads": heads, "useful_flop_per_tile": 2 * 128 * heads * (576 + 512)}
+        for form, fname in ((0, "transposed"), (1, "untransposed")):
+            for streams, sname in ((1, "scores"), (2, "output"), (3, "both")):
+                for _ in range(2):  # the first launch warms the clocks and the instruction cache
+                    mla.mla_form_ablation(form, heads, streams, tiles, cycles, err)
+                torch.cuda.synchronize()
+                if int(err.item()) != 0:
+                    raise RuntimeError("form ablation: a bounded wait ran out")
+                cyc = cycles.max().item() / tiles
+                entry[f"{fname}_{sname}_cycles_per_tile"] = round(cyc, 1)
+            entry[f"{fname}_useful_flop_per_cycle_per_sm"] = round(
+                entry["useful_flop_per_tile"] / entry[f"{fname}_both_cycles_per_tile"], 1)
+        entry["untransposed_over_transposed"] = round(entry["untransposed_both_cycles_per_tile"] /
+                                                      entry["transposed_both_cycles_per_tile"], 3)
+        rows.append(entry)
+    print(json.dumps({"ablation": "transposed vs untransposed MMAs per 128-row KV tile, bf16, d_qk 576, d_v 512",
+                      "ctas": ctas, "tiles_per_cta": tiles, "rows": rows}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -561,11 +594,15 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="b16_h16_64k")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--ablation", action="store_true",
+                    help="print the transposed-vs-untransposed tensor-core cost table instead of a bench line")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-rows", type=int, default=4096)
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
+    if args.ablation:
+        return run_ablation(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

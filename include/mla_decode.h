@@ -193,6 +193,23 @@ MLA_API int mla_combine(const void *workspace, int batch, int q_len, int num_hea
 MLA_API int mla_stream_probe(const void *kv, int64_t rows, int units, int32_t *err, void *stream);
 
 /*
+ * Measurement helper for the pages' argument for the transposed form (FlashMLA-ETAP technical
+ * summary, "Problem Statement": with few heads the untransposed S = Q K^T pads the query heads up
+ * to the tensor core's minimum M; "Methodology": S^T = K Q^T puts the KV rows on M instead).  Issues,
+ * on each of `ctas` CTAs, the tensor-core instructions of `tiles` 128-row KV tiles for h = `heads`
+ * query heads (d_qk 576, d_v 512, bf16 operands, fp32 accumulators) in one form:
+ *   form 0 transposed:   S^T M=128 N=h K=576; O^T 4 x (M=128 N=h K=128)
+ *   form 1 untransposed: S M=hpad N=128 K=576; O 2 x (M=hpad N=256 K=128), hpad = 64 (h <= 64) or 128
+ * streams: 1 the score MMAs only, 2 the output MMAs only, 3 both (from two issuing threads).
+ * cycles: device [ctas] uint64, written with each CTA's clock cycles from the first issue to the
+ * completion of its last MMA.  err: device int32, zeroed by the caller, set to 1 if the bounded wait
+ * for completion ran out.  The operands are zero-filled shared memory (no data is read from or
+ * written to global memory besides these two).  Asynchronous on `stream`; allocates nothing.
+ */
+MLA_API int mla_form_ablation(int form, int heads, int streams, int tiles, int ctas, unsigned long long *cycles,
+                      int32_t *err, void *stream);
+
+/*
  * Copy the workspace status word to the host (waits for that copy only).
  * *status_out receives MLA_OK or the first device-side error recorded.
  */

@@ -28,7 +28,7 @@ STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3:
 
 EXPORTS = ("mla_decode_workspace_size", "mla_decode_plan", "mla_decode_fwd", "mla_combine",
            "mla_decode_read_status", "mla_decode_plan_host", "mla_status_string", "mla_last_cuda_error",
-           "mla_decode_fwd_static_ws", "mla_decode_fwd_ragged", "mla_stream_probe", "mla_decode_fwd_fp8")
+           "mla_decode_fwd_static_ws", "mla_decode_fwd_ragged", "mla_stream_probe", "mla_decode_fwd_fp8", "mla_form_ablation")
 STATIC_WORKSPACE_BYTES = 8388608
 
 
@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_fwd_static_ws.argtypes = [vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp,
                                                vp, i32, vp]
         L.mla_decode_fwd_static_ws.restype = i32
+        L.mla_form_ablation.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp]
+        L.mla_form_ablation.restype = i32
         L.mla_stream_probe.argtypes = [vp, i64, i32, vp, vp]
         L.mla_stream_probe.restype = i32
         L.mla_last_cuda_error.argtypes = []
@@ -161,6 +163,13 @@ def mla_stream_probe(kv, units: int, err, stream=None) -> None:
     no computation (a bandwidth probe).  ``err``: int32 device tensor [1], zeroed by the caller."""
     rows = kv.numel() // 576
     _check(lib().mla_stream_probe(_ptr(kv), rows, units, _ptr(err), _stream(stream)), "mla_stream_probe")
+
+
+def mla_form_ablation(form: int, heads: int, streams: int, tiles: int, cycles, err, stream=None) -> None:
+    """Tensor-core instructions of ``tiles`` KV tiles per CTA in the transposed (form 0) or untransposed
+    (form 1) layout; ``cycles``: uint64-compatible int64 device tensor [ctas], ``err``: int32 [1] zeroed."""
+    _check(lib().mla_form_ablation(form, heads, streams, tiles, cycles.numel(), _ptr(cycles), _ptr(err),
+                                   _stream(stream)), "mla_form_ablation")
 
 
 def mla_combine(workspace, batch, q_len, num_heads, n_sms, o, lse, stream=None) -> None:

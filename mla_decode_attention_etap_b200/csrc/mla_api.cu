@@ -16,6 +16,7 @@
 #include "etap_pair_kernel.cuh"
 #include "plan_combine_kernels.cuh"
 #include "plan_core.h"
+#include "form_ablation.cuh"
 #include "stream_probe.cuh"
 
 namespace {
@@ -396,6 +397,28 @@ int mla_stream_probe(const void *kv, int64_t rows, int units, int32_t *err, void
     mla::stream_probe_kernel<<<2 * units, 64, mla::kProbeSmem, s>>>(tm_kv, tm_kvr, pp);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "stream_probe_kernel launch");
+    return MLA_OK;
+}
+
+int mla_form_ablation(int form, int heads, int streams, int tiles, int ctas, unsigned long long *cycles, int32_t *err,
+                      void *stream) {
+    if (form != 0 && form != 1) return MLA_ERR_INVALID_ARG;
+    if (heads != 16 && heads != 32 && heads != 64 && heads != 128) return MLA_ERR_INVALID_ARG;
+    if (streams < 1 || streams > 3 || tiles < 1 || tiles > 65536 || ctas < 1 || ctas > 4096) return MLA_ERR_INVALID_ARG;
+    if (!cycles || !err) return MLA_ERR_INVALID_ARG;
+    if (!aligned(cycles, 8) || !aligned(err, 4)) return MLA_ERR_ALIGNMENT;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(mla::form_ablation_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)mla::kAblSmem);
+    });
+    if (attr_err != cudaSuccess) return cuda_fail(attr_err, "cudaFuncSetAttribute");
+    mla::AblationParams ap{form, heads, streams, tiles, cycles, err};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    mla::form_ablation_kernel<<<ctas, 64, mla::kAblSmem, s>>>(ap);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "form_ablation_kernel launch");
     return MLA_OK;
 }
 

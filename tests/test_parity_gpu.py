@@ -380,3 +380,20 @@ def test_append_ragged_paged():
 def test_full_b16_h16_append_q16_sampled():
     w = W.workload_b16_h16_append_q16(seed=0, device="cuda")
     _full(w, [0, 9])
+
+
+@pytest.mark.parametrize("heads", [16, 64, 128])
+def test_form_ablation_runs(heads):
+    """The transposed/untransposed tensor-core ablation completes on every form and stream choice."""
+    import mla_decode_attention_etap_b200 as mla
+    dev = torch.device("cuda")
+    cycles = torch.zeros(4, dtype=torch.int64, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    for form in (0, 1):
+        for streams in (1, 2, 3):
+            cycles.zero_()
+            mla.mla_form_ablation(form, heads, streams, 8, cycles, err)
+            torch.cuda.synchronize()
+            assert int(err.item()) == 0
+            # at least 8 tiles x 16 MMAs at >= 8 cycles each
+            assert int(cycles.min().item()) > 8 * 16 * 8
