@@ -73,6 +73,8 @@ struct PairCfg {
     // after the barrier that ends the tile, instead of handing P^T to the MMA warp (its polling and
     // the score MMAs it may be issuing would delay it); the issuing warp has a tile's time to spare.
     static constexpr bool PV_BY_SOFTMAX = CH == 1;
+    // threads that issue step 3 (one V slot each; E4M3: two, so that neither blocks for a whole tile)
+    static constexpr int PV_SPLIT = KV8 ? 2 : 1;
     static constexpr int PREFETCH = 1;                                 // tiles the L2 prefetch runs ahead of the loads
     static constexpr uint32_t CHUNK = 16384;                           // 128 rows x 128 bytes, 128B swizzle
     static constexpr uint32_t HALF = 8192;                             // 64 rows of a chunk = one TMA box
@@ -216,11 +218,11 @@ __global__ void __launch_bounds__(320, 1)
         }
         for (int i = 0; i < C::PB; ++i) {
             mbar_init(bar(BR::PFULL + i), 8);
-            mbar_init(bar(BR::PEMPTY + i), 1);
+            mbar_init(bar(BR::PEMPTY + i), C::PV_BY_SOFTMAX ? C::PV_SPLIT : 1);
         }
         mbar_init(bar(BR::TAIL), 1);
         mbar_init(bar(BR::FINAL), 1);
-        mbar_init(bar(BR::SFIN), 1);
+        mbar_init(bar(BR::SFIN), C::PV_SPLIT);
         mbar_init(bar(BR::RED), 4);
         mbar_init(bar(BR::REDL), 4);
         for (int i = 0; i < 8 * C::XS; ++i) mbar_init(bar(BR::XFULL + i), 1);
@@ -247,10 +249,11 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tmem = *tmem_slot;
     // Step 3 of tile kk: O^T (+)= V^T P^T for the CTA's 256 latent rows (two M-tiles); frees each
     // V slot and then the P^T buffer as the MMAs complete.
-    auto issue_pv = [&](int kk, bool first) {
+    // part: which V slots (all with PV_SPLIT == 1); every issuing part commits PEMPTY once.
+    auto issue_pv = [&](int kk, bool first, int part) {
         const int pb = kk % C::PB;
         const uint32_t p_base = sbase + C::OFF_P + pb * C::P_BUF;
-        for (int i = 0; i < C::PAIRS; ++i) {
+        for (int i = part * C::PAIRS / C::PV_SPLIT; i < (part + 1) * C::PAIRS / C::PV_SPLIT; ++i) {
             const int g2 = C::PAIRS * kk + i;
             const int vs = g2 % C::NV;
             const uint32_t v_base = sbase + C::OFF_V + vs * C::V_SLOT;
@@ -519,7 +522,7 @@ __global__ void __launch_bounds__(320, 1)
                 if constexpr (!C::PV_BY_SOFTMAX) {
                     if (kp < kq && mbar_test_wait(bar(BR::PFULL + kp % C::PB), (kp / C::PB) & 1)) {
                         tc_fence_after();
-                        issue_pv(kp, pc.first());
+                        issue_pv(kp, pc.first(), 0);
                         pc.advance(tile_off);
                         ++kp;
                         progressed = true;
@@ -1034,9 +1037,9 @@ __global__ void __launch_bounds__(320, 1)
                     if constexpr (C::PV_BY_SOFTMAX) {
                         // every P^T row written and every O^T rescale done: one thread issues step 3
                         named_bar_sync(SMX, NSM);
-                        if (warp == 2 && lane == 0) {
+                        if (lane == 0 && (warp == 2 || (C::PV_SPLIT == 2 && warp == 6))) {
                             tc_fence_after();
-                            issue_pv(k, first);
+                            issue_pv(k, first, warp == 2 ? 0 : 1);
                             pv_issued = true;
                         }
                     } else {
