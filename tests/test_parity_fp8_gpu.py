@@ -171,3 +171,44 @@ def test_unsupported_column_count_is_rejected():
     with pytest.raises(MlaError) as ei:
         dec.fwd_fp8(w.q.to(dev), w.kv8.to(dev), w.kv_scale.to(dev), sl)
     assert ei.value.code == -2
+
+
+def test_bounded_waits_report_timeout_and_context_survives():
+    """Failure detection without a GPU fault on the FP8 path: with the quantised Q withheld the
+    bounded waits run out, the status word says MLA_ERR_TIMEOUT, and the next call is correct."""
+    from mla_decode_attention_etap_b200 import FLAG_TEST_EXPIRE_WAITS
+    w = fp8(2, 16, [3000, 700], seed=111)
+    _, _, st, dec = run_cuda(w, flags=FLAG_TEST_EXPIRE_WAITS, poison=False)
+    assert st == -6  # MLA_ERR_TIMEOUT
+    o, lse, st2, _ = run_cuda(w, decoder=dec)
+    assert st2 == 0
+    assert_parity(o, lse, *run_oracle(w), what="fp8 after an expired wait")
+
+
+def test_cuda_graph_replay_matches_eager():
+    """plan + FP8 decode captured in a CUDA graph and replayed: bitwise the eager result."""
+    w = fp8(3, 16, [5000, 700, 2100], seed=112)
+    dev = torch.device("cuda")
+    q, kv8, sc, sl = w.q.to(dev), w.kv8.to(dev), w.kv_scale.to(dev), w.seqlens.to(dev)
+    dec = MlaDecoder(w.batch, w.q_len, w.num_heads, device=dev)
+    o = torch.empty(w.batch, 1, 16, 512, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(w.batch, 1, 16, dtype=torch.float32, device=dev)
+    dec.plan(sl)
+    dec.fwd_fp8(q, kv8, sc, sl, None, w.softmax_scale, False, o=o, lse=lse)
+    torch.cuda.synchronize()
+    o_eager, l_eager = o.clone(), lse.clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            dec.plan(sl, stream=side)
+            dec.fwd_fp8(q, kv8, sc, sl, None, w.softmax_scale, False, o=o, lse=lse, stream=side)
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(3):
+        o.zero_()
+        lse.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(o, o_eager) and torch.equal(lse, l_eager)
+    assert dec.status() == 0
