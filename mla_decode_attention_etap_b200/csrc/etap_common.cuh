@@ -56,7 +56,7 @@ struct DecodeParams {
     float scale_log2;  // softmax_scale * log2(e)
     unsigned long long wait_limit_ns;
     int withhold_q;    // test hook: never load Q, so that the bounded waits expire
-    int cta_ranges_off, tile_off_off, seq_info_off;  // int32 offsets into ws
+    int cta_ranges_off, tile_off_off, seq_info_off, cta_seq_off;  // int32 offsets into ws
     int32_t *counters;  // [batch][groups][2]: split CTAs done per (sequence, column group, rank)
     int slots;          // partial slots (stride between the two ranks' LSE partial arrays)
     int fuse_merge;     // the last split CTA of a sequence merges the partials (no combine launch)
@@ -109,6 +109,12 @@ struct SegIter {
         }
         b = lo;
     }
+    // Same, starting from the sequence b0 that holds tile fb (from the plan): no search.
+    __device__ void init_at(int b0, int64_t fb, int64_t fe_) {
+        f = fb;
+        fe = fe_;
+        b = b0;
+    }
     __device__ bool next(const int32_t *tile_off, int &ob, int &t0, int &t1) {
         if (f >= fe) return false;
         while (tile_off[b + 1] <= f) ++b;
@@ -137,8 +143,8 @@ struct TileCursorT {
             }
         }
     }
-    __device__ void init(const int32_t *tile_off, int batch, int64_t fb, int64_t fe, int off_ = 0) {
-        it.init(tile_off, batch, fb, fe);
+    __device__ void init(const int32_t *tile_off, int b0, int64_t fb, int64_t fe, int off_ = 0) {
+        it.init_at(b0, fb, fe);
         off = STEP > 1 ? off_ : 0;
         b = t0 = t = t1 = 0;
         valid = it.next(tile_off, b, t0, t1);

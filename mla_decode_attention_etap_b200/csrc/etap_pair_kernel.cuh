@@ -302,6 +302,7 @@ __global__ void __launch_bounds__(320, 1)
     const int32_t *tile_off = p.ws + p.tile_off_off;
     const int32_t *seq_info = p.ws + p.seq_info_off;
     const int64_t fb = plan_ok ? ranges[2 * unit] : 0, fe = plan_ok ? ranges[2 * unit + 1] : 0;
+    const int seq0 = plan_ok ? p.ws[p.cta_seq_off + unit] : 0;  // the sequence holding tile fb
     if (!plan_ok && threadIdx.x == 0) atomicCAS(status, 0, kStatusInvalid);
     const int64_t l_cap = p.paged ? (int64_t)p.max_blocks * kPage : p.kv_rows;
     // first rope column of this CTA (E4M3: all 64 rope columns, every CTA)
@@ -345,7 +346,7 @@ __global__ void __launch_bounds__(320, 1)
         };
         TileCursorT<C::TSTEP> ahead;
         if (fb < fe && lane == 0) {
-            ahead.init(tile_off, p.batch, fb, fe, toff);
+            ahead.init(tile_off, seq0, fb, fe, toff);
             for (int d = 0; d < C::PREFETCH && ahead.valid; ++d) {
                 prefetch_tile(ahead.b, ahead.t);
                 ahead.advance(tile_off);
@@ -353,7 +354,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (fb < fe) {
             SegIter it;
-            it.init(tile_off, p.batch, fb, fe);
+            it.init_at(seq0, fb, fe);
             int b, t0, t1, seg = 0, k = 0;
             while (ok && it.next(tile_off, b, t0, t1)) {
                 int L = p.seqlens[b];
@@ -511,8 +512,8 @@ __global__ void __launch_bounds__(320, 1)
                 }
             };
             TileCursorT<C::TSTEP> qc, pc;
-            qc.init(tile_off, p.batch, fb, fe, toff);
-            pc.init(tile_off, p.batch, fb, fe, toff);
+            qc.init(tile_off, seq0, fb, fe, toff);
+            pc.init(tile_off, seq0, fb, fe, toff);
             int kq = 0, kp = 0, seg_q = 0;
             int qstage = 0;  // scores of tile kq: 0 = rope columns next, 1 + i = V pair i next
             uint64_t t_last = global_timer_ns();
@@ -635,7 +636,7 @@ __global__ void __launch_bounds__(320, 1)
         };
         if (fb < fe) {
             SegIter it;
-            it.init(tile_off, p.batch, fb, fe);
+            it.init_at(seq0, fb, fe);
             int b, t0, t1, k = 0, seg = 0, e = 0, red_uses = 0;
             int qseg = 0;  // E4M3: segments with a tile for this CTA (Q operands written so far)
             int mseg = 0;  // E4M3: segment merges with the peer so far

@@ -333,6 +333,7 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
     p.cta_ranges_off = (int)(lay.cta_ranges / 4);
     p.tile_off_off = (int)(lay.tile_off / 4);
     p.seq_info_off = (int)(lay.seq_info / 4);
+    p.cta_seq_off = (int)(lay.cta_seq / 4);
     p.counters = reinterpret_cast<int32_t *>(ws + lay.counters);
     p.slots = lay.slots;
     // splits of a sequence are at most the work units (CTA pairs per column group)

@@ -56,6 +56,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t *__res
     int32_t *ranges = ws + lay.cta_ranges / 4;
     int32_t *seq_info = ws + lay.seq_info / 4;
     int32_t *counters = ws + lay.counters / 4;
+    int32_t *cta_seq = ws + lay.cta_seq / 4;
     const int per = (batch + kPlanThreads - 1) / kPlanThreads;
     const int b0 = min(batch, (int)threadIdx.x * per), b1 = min(batch, b0 + per);
     // flattened tile offsets: exclusive prefix sum of tiles per sequence
@@ -74,6 +75,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t *__res
             nsplit = cta_of(total, used, t1 - 1) - first + 1;
         }
         tile_off[b] = (int32_t)t0;
+        // the units whose range starts inside this sequence start their walk here
+        for (int c = first; c >= 0 && c < first + nsplit; ++c)
+            if (cta_begin(total, used, c) >= t0) cta_seq[c] = b;
         seq_info[4 * b + 0] = (int32_t)(t1 - t0);
         seq_info[4 * b + 1] = first;
         seq_info[4 * b + 2] = nsplit;
@@ -90,6 +94,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t *__res
     for (int c = threadIdx.x; c < ctas; c += kPlanThreads) {
         ranges[2 * c] = (int32_t)cta_begin(total, used, c);
         ranges[2 * c + 1] = (int32_t)cta_begin(total, used, c + 1);
+        if (c >= used) cta_seq[c] = batch;  // no tiles
     }
     for (int i = threadIdx.x; i < 2 * batch * groups; i += kPlanThreads) counters[i] = 0;
     if (threadIdx.x == 0) {

@@ -64,6 +64,7 @@ MLA_HD size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct WsLayout {
     size_t cta_ranges;  // int32 [ctas][2] (one range per work unit = SM pair)
+    size_t cta_seq;     // int32 [ctas]: the sequence that holds the unit's first tile (batch if none)
     size_t tile_off;    // int32 [batch + 1]
     size_t seq_info;    // int32 [batch][4]: tiles, first CTA, splits, slot offset
     size_t opart;       // fp32  [slots][ncols][512]
@@ -82,6 +83,8 @@ MLA_HD WsLayout ws_layout(int batch, int q_len, int num_heads, int num_sms) {
     size_t off = align256(sizeof(int32_t) * kHdrWords);
     w.cta_ranges = off;
     off += align256(sizeof(int32_t) * 2 * (size_t)w.ctas);
+    w.cta_seq = off;
+    off += align256(sizeof(int32_t) * (size_t)w.ctas);
     w.tile_off = off;
     off += align256(sizeof(int32_t) * ((size_t)batch + 1));
     w.seq_info = off;

@@ -262,13 +262,18 @@ def test_device_plan_matches_host_plan(batch):
     ranges, info, nct, _ = mla_decode_plan_host(lens, 1, 16, dec.n_sms)
     ws = dec.workspace.view(torch.int32).cpu().numpy()
     off_ranges = _a256(4 * 64)
-    off_tile = off_ranges + _a256(4 * 2 * nct)
+    off_seq = off_ranges + _a256(4 * 2 * nct)
+    off_tile = off_seq + _a256(4 * nct)
     off_info = off_tile + _a256(4 * (batch + 1))
     np.testing.assert_array_equal(ws[off_ranges // 4: off_ranges // 4 + 2 * nct].reshape(-1, 2), ranges)
     np.testing.assert_array_equal(ws[off_info // 4: off_info // 4 + 4 * batch].reshape(-1, 4), info)
     tiles = (lens.astype(np.int64) + 127) // 128
-    np.testing.assert_array_equal(ws[off_tile // 4: off_tile // 4 + batch + 1],
-                                  np.concatenate([[0], np.cumsum(tiles)]).astype(np.int32))
+    tile_off = np.concatenate([[0], np.cumsum(tiles)]).astype(np.int64)
+    np.testing.assert_array_equal(ws[off_tile // 4: off_tile // 4 + batch + 1], tile_off.astype(np.int32))
+    # each unit's first sequence: the one whose tile range holds the unit's first tile (batch if none)
+    want = np.array([int(np.searchsorted(tile_off, fb, side="right") - 1) if fb < fe else batch
+                     for fb, fe in ranges], dtype=np.int32)
+    np.testing.assert_array_equal(ws[off_seq // 4: off_seq // 4 + nct], want)
     assert ws[0] == 0 and ws[1] == nct and ws[3] == batch and ws[4] == int(tiles.sum())
 
 
