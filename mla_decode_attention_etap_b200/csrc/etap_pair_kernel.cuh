@@ -69,12 +69,12 @@ struct PairCfg {
     static constexpr int XS = CH > 2 ? CH : 2;                         // exchange slots (8 KB each)
     // KV8: the segment merge receives 2 M-tiles x 128 rows x 16 fp32 plus 16 (m, l) per softmax warp
     static constexpr uint32_t X_BYTES = KV8 ? 2 * 128 * 16 * 4 + 8 * 16 * 4 : XS * 128 * 16 * 4;
-    // One column chunk per thread (h*q_len <= 16): the softmax warps issue step 3 themselves, right
-    // after the barrier that ends the tile, instead of handing P^T to the MMA warp (its polling and
-    // the score MMAs it may be issuing would delay it); the issuing warp has a tile's time to spare.
-    static constexpr bool PV_BY_SOFTMAX = CH == 1;
-    // threads that issue step 3 (one V slot each; E4M3: two, so that neither blocks for a whole tile)
-    static constexpr int PV_SPLIT = KV8 ? 2 : 1;
+    // The softmax warps issue step 3 themselves, right after the barrier that ends the tile, instead
+    // of handing P^T to the MMA warp (its polling and the score MMAs it may be issuing would delay
+    // it); for 32-column groups and the E4M3 cache two threads share it, one V slot each.
+    static constexpr bool PV_BY_SOFTMAX = CH <= 2;
+    // threads that issue step 3 (one V slot each when two, so that neither blocks for a whole tile)
+    static constexpr int PV_SPLIT = (KV8 || CH == 2) ? 2 : 1;
     static constexpr int PREFETCH = 1;                                 // tiles the L2 prefetch runs ahead of the loads
     static constexpr uint32_t CHUNK = 16384;                           // 128 rows x 128 bytes, 128B swizzle
     static constexpr uint32_t HALF = 8192;                             // 64 rows of a chunk = one TMA box
