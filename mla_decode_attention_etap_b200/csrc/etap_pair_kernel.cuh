@@ -22,15 +22,15 @@
 //     two 64-column chunks plus 8 KB slots for the 32 rope columns; tail rows
 //     zeroed; L2 prefetch one tile ahead);
 //   * warp 1 lane 0: tcgen05.mma issuer, an event loop over the score MMAs of
-//     the next tile (in stages, as their operands land) and, for 32-column
-//     groups, O^T of the oldest tile whose P^T is ready (for 16 columns one
-//     softmax thread issues O^T right after the barrier that ends the tile);
+//     the next tile (in stages, as their operands land);
 //   * warps 2..9: two warps per TMEM lane quadrant, one KV row and half of the
 //     columns per thread; the column softmax reduces ACROSS threads; P^T goes
-//     to shared memory as bf16 hi | lo; at the end of a split the last CTA of
-//     a sequence merges the split partials (log-sum-exp).
+//     to shared memory as bf16 hi | lo; one or two softmax threads issue O^T
+//     right after the barrier that ends the tile; at the end of a split the
+//     last CTA of a sequence merges the split partials (log-sum-exp).
 //
-// Every wait is bounded; see etap_common.cuh.
+// The E4M3-cache configuration (PairCfg16E4) keeps the roles but not the column
+// split: see PairCfg.  Every wait is bounded; see etap_common.cuh.
 #pragma once
 
 #include "etap_common.cuh"
