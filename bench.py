@@ -7,14 +7,17 @@ ETAP decode kernel (which also merges the split-KV partials, log-sum-exp).  Defa
 latent KV, larger than the 126 MB L2, so no flush is needed between steps).
 
 Reported value: whole-job KV throughput in TB/s (algorithmic bytes: 1152 per
-cached token read once) over the max-over-ranks device time of K steps.  The
-line also carries TFLOPS (2*(576+512) flops per visible (query column, token)
-pair), the decode kernel's roofline fraction (live CUDA-event timing of that
-kernel on its stream), an end-to-end figure through the C ABI with host
-buffers, the fp64 oracle timed on the host as a CPU baseline, and GPU clocks
-sampled while the steps run.
+cached token read once, 580 for the FP8 cache) over the max-over-ranks device
+time of K steps, replayed from CUDA graphs of the same calls (--no-graph launches
+them from the host).  The line also carries TFLOPS (2*(576+512) flops per visible
+(query column, token) pair), the decode kernel's roofline fraction (CUDA-event
+timing of back-to-back launches of that kernel on its stream, taken right before
+the timed steps), an end-to-end figure through the C ABI with host buffers, the
+fp64 oracle timed on the host as a CPU baseline, and GPU clocks sampled while the
+steps run.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+  python bench.py --ablation    # transposed vs untransposed tensor-core cost per KV tile
 
 N > 1 runs under torchrun, one process per GPU; every rank decodes its own
 batch (independent sequences, no collective on the data path: weak scaling).
