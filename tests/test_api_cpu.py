@@ -100,3 +100,49 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(ImportError):
         m.lib()
+
+
+def fwd_fp8(**kw):
+    args = dict(q=A, kv8=A, kv_scale=A, seqlens=A, q_lens=None, block_table=None, batch=2, q_len=1, num_heads=16,
+                kv_rows=128, max_blocks=0, scale=1 / 24, causal=0, o=A, lse=A, ws=A, ws_bytes=1 << 30, n_sms=148,
+                flags=0)
+    args.update(kw)
+    vp = ctypes.c_void_p
+    opt = lambda x: vp(x) if x else None  # noqa: E731
+    return m.lib().mla_decode_fwd_fp8(vp(args["q"]), opt(args["kv8"]), opt(args["kv_scale"]), vp(args["seqlens"]),
+                                      opt(args["q_lens"]), opt(args["block_table"]), args["batch"], args["q_len"],
+                                      args["num_heads"], args["kv_rows"], args["max_blocks"],
+                                      ctypes.c_float(args["scale"]), args["causal"], vp(args["o"]), vp(args["lse"]),
+                                      vp(args["ws"]), args["ws_bytes"], args["n_sms"], args["flags"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(kv_scale=0), -1),                     # the FP8 entry needs its row scales
+    (dict(kv8=0), -1),
+    (dict(num_heads=32), -2), (dict(q_len=2), -2),   # more than 16 query columns
+    (dict(scale=0.0), -1), (dict(causal=3), -1),
+    (dict(kv8=A + 8), -3), (dict(kv_scale=A + 2), -3), (dict(q_lens=A + 2), -3),
+    (dict(ws_bytes=100), -4),
+])
+def test_fwd_fp8_rejects(kw, code):
+    assert fwd_fp8(**kw) == code
+
+
+def test_measurement_helpers_reject():
+    L = m.lib()
+    vp = ctypes.c_void_p
+    ok = dict(form=0, heads=16, streams=3, tiles=8, ctas=2, cycles=A, err=A)
+
+    def abl(**kw):
+        a = dict(ok, **kw)
+        return L.mla_form_ablation(a["form"], a["heads"], a["streams"], a["tiles"], a["ctas"],
+                                   vp(a["cycles"]) if a["cycles"] else None, vp(a["err"]) if a["err"] else None,
+                                   None)
+    for kw in (dict(form=2), dict(heads=48), dict(streams=0), dict(streams=4), dict(tiles=0), dict(ctas=0),
+               dict(cycles=0), dict(err=0)):
+        assert abl(**kw) == -1, kw
+    assert abl(cycles=A + 4) == -3
+    assert abl(err=A + 2) == -3
+    assert L.mla_stream_probe(vp(A), 100, 74, vp(A), None) == -1      # rows not a multiple of 128
+    assert L.mla_stream_probe(vp(A), 256, 0, vp(A), None) == -1
+    assert L.mla_stream_probe(vp(A + 8), 256, 74, vp(A), None) == -3
