@@ -68,6 +68,8 @@ WORKLOADS = {
     "b16_h16_16k_fp8": dict(batch=16, heads=16, seqlen=16384, fp8=True),
     "b16_h16_4k_fp8": dict(batch=16, heads=16, seqlen=4096, fp8=True),
     "b64_h16_paged_fp8": dict(kind="b64_paged_fp8"),
+    "b16_h16_q4_causal_fp8": dict(kind="q4_causal_fp8"),
+    "b32_h128_paged_fp8": dict(kind="b32_h128_fp8"),
 }
 
 
@@ -120,6 +122,14 @@ def make_workload(name: str, rank: int, device):
     if kind == "append_q16":
         return (W.workload_b16_h16_append_q16(seed=seed, device=device),
                 "mla_decode_b16_h16_append_q16_causal_L32768")
+    if kind == "q4_causal_fp8":
+        return (W.make_workload(16, 16, [32768] * 16, q_len=4, causal=True, seed=seed, device=device,
+                                spike_frac=0.05, spike_scale=8.0, kv_dtype="e4m3"),
+                "mla_decode_b16_h16_q4_causal_L32768_spikes5pct_x8_e4m3cache")
+    if kind == "b32_h128_fp8":
+        lens = W.draw_seqlens(32, 8192, 32768, seed)
+        return (W.make_workload(32, 128, lens, paged=True, seed=seed, device=device, kv_dtype="e4m3"),
+                "mla_decode_b32_h128_q1_Lunif8192to32768_paged64_e4m3cache")
     if kind == "b64_paged_fp8":
         return (W.workload_b64_h16_paged_fp8(seed=seed, device=device),
                 "mla_decode_b64_h16_q1_Lunif1to65536_paged64_e4m3cache")

@@ -162,10 +162,11 @@ MLA_API int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *
  *              or [kv_rows / 64, 64]), 4-byte aligned, must not be NULL; a scale must be
  *              finite and >= 0 (values below 2^-100 count as 2^-100 in the maximum)
  *   q_lens     as for mla_decode_fwd_ragged, or NULL
- * Supported for q_len * num_heads <= 16 (else MLA_ERR_UNSUPPORTED).  The kernel
- * stores Q per query column as two E4M3 terms times a power of two, and P as two
- * E4M3 terms; the fp32 accumulation, the split-KV merge and the outputs are those
- * of mla_decode_fwd.  All other arguments, layouts and errors as there.
+ * Any q_len * num_heads up to MLA_MAX_COLUMNS, in groups of 16 or 32 query columns
+ * as for mla_decode_fwd.  The kernel stores Q per query column as two E4M3 terms
+ * times a power of two, and P as two E4M3 terms; the fp32 accumulation, the
+ * split-KV merge and the outputs are those of mla_decode_fwd.  All other
+ * arguments, layouts and errors as there.
  */
 MLA_API int mla_decode_fwd_fp8(const void *q, const void *kv8, const float *kv_scale, const int32_t *seqlens,
                        const int32_t *q_lens, const int32_t *block_table, int batch, int q_len, int num_heads,

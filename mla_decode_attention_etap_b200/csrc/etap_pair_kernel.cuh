@@ -67,8 +67,12 @@ struct PairCfg {
     static constexpr int CHUNK_COLS = KV8 ? 128 : 64;
     static constexpr int VCOLS = KV8 ? 512 : 256;  // latent (V) columns of a tile this CTA loads
     static constexpr int XS = CH > 2 ? CH : 2;                         // exchange slots (8 KB each)
-    // KV8: the segment merge receives 2 M-tiles x 128 rows x 16 fp32 plus 16 (m, l) per softmax warp
-    static constexpr uint32_t X_BYTES = KV8 ? 2 * 128 * 16 * 4 + 8 * 16 * 4 : XS * 128 * 16 * 4;
+    // bf16: the per-tile score exchange slots.  E4M3: none; the segment merge receives 2 M-tiles x
+    // 128 rows x NG fp32 plus NG/2 (m, l) pairs per softmax warp into the Q and P^T area, idle by then.
+    static constexpr uint32_t X_BYTES = KV8 ? 0 : XS * 128 * 16 * 4;
+    static constexpr uint32_t XM_ROW = NG * 4;                          // bytes per row of a merge M-tile
+    static constexpr uint32_t XM_TILE = 128 * XM_ROW;
+    static constexpr uint32_t XM_BYTES = 2 * XM_TILE + 8 * NG * 4;
     // The softmax warps issue step 3 themselves, right after the barrier that ends the tile, instead
     // of handing P^T to the MMA warp (its polling and the score MMAs it may be issuing would delay
     // it); for 32-column groups and the E4M3 cache two threads share it, one V slot each.
@@ -107,6 +111,10 @@ struct PairCfg {
     static constexpr uint32_t OFF_QR = OFF_Q + Q_CHUNKS * Q_CHUNK;
     static constexpr uint32_t OFF_P = align1024(OFF_QR + Q_ROPE);
     static constexpr uint32_t OFF_X = OFF_P + PB * P_BUF;
+    static constexpr uint32_t OFF_XM = KV8 ? OFF_Q : OFF_X;            // E4M3: segment-merge receive area
+    // the in-kernel split merge stages (splits + 1) x NG floats: E4M3 in the Q area, else in the P^T buffers
+    static constexpr uint32_t OFF_STAGE = KV8 ? OFF_Q : OFF_P;
+    static constexpr uint32_t STAGE_BYTES = KV8 ? OFF_P - OFF_Q : PB * P_BUF;
     static constexpr uint32_t OFF_BAR = OFF_X + X_BYTES;
     static constexpr uint32_t OFF_RED = OFF_BAR + 512;                 // float [2][4][NG] column max exchange
     static constexpr uint32_t OFF_REDL = OFF_RED + 32 * NG;               // float [4][NG] column sum exchange
@@ -122,20 +130,25 @@ struct PairCfg {
     static constexpr float THRESH = KV8 ? kRescaleThreshold8 : kRescaleThreshold;
     static constexpr float HEADROOM = KV8 ? kRescaleHeadroom8 : kRescaleHeadroom;
     // The in-kernel split merge stages (splits + 1) x NG floats in the idle P^T buffers.
-    static constexpr int MERGE_MAX_SPLITS = (int)(PB * P_BUF / 4) / NG - 1;
+    static constexpr int MERGE_MAX_SPLITS = (int)(STAGE_BYTES / 4) / NG - 1;
 };
 
 using PairCfg16 = PairCfg<16, 5, 2, 2>;  // h*q_len <= 16
 using PairCfg32 = PairCfg<32, 5, 1, 1>;  // 16 < h*q_len, in groups of 32 columns
 // E4M3 cache, h*q_len <= 16: whole tiles per CTA, 2.5 tiles in flight
 using PairCfg16E4 = PairCfg<16, 5, 2, 2, true>;
+// E4M3 cache, groups of 32 columns: one P^T buffer (N = 64, 8 KB)
+using PairCfg32E4 = PairCfg<32, 5, 2, 1, true>;
 
 template <class C>
 constexpr bool pair_cfg_fits() {
     return C::SMEM_ALLOC <= 232448 && C::TMEM_COLS <= 512 && C::OFF_P % 1024 == 0 && C::OFF_QR % 512 == 0 &&
-           C::OFF_R % 1024 == 0 && C::R_SLOT % 256 == 0 && C::OFF_Q % 1024 == 0 && (!C::KV8 || C::CH == 1);
+           C::OFF_R % 1024 == 0 && C::R_SLOT % 256 == 0 && C::OFF_Q % 1024 == 0 && (!C::KV8 || C::CH <= 2) &&
+           (!C::KV8 || (C::OFF_P + C::PB * C::P_BUF - C::OFF_Q >= C::XM_BYTES &&
+                        C::OFF_P == C::OFF_Q + 4 * C::Q_CHUNK + C::Q_ROPE));
 }
-static_assert(pair_cfg_fits<PairCfg16>() && pair_cfg_fits<PairCfg32>() && pair_cfg_fits<PairCfg16E4>(),
+static_assert(pair_cfg_fits<PairCfg16>() && pair_cfg_fits<PairCfg32>() && pair_cfg_fits<PairCfg16E4>() &&
+                  pair_cfg_fits<PairCfg32E4>(),
               "shared memory / TMEM plan");
 
 template <class C>
@@ -163,7 +176,7 @@ struct PairBars {
     static constexpr int COUNT = XFREE + 8;
 };
 static_assert(PairBars<PairCfg16>::COUNT * 8 <= 512 && PairBars<PairCfg32>::COUNT * 8 <= 512 &&
-                  PairBars<PairCfg16E4>::COUNT * 8 <= 512,
+                  PairBars<PairCfg16E4>::COUNT * 8 <= 512 && PairBars<PairCfg32E4>::COUNT * 8 <= 512,
               "barrier area");
 
 // Byte offset of 16-byte chunk j of row r in a row-major buffer of `pitch`-byte
@@ -686,22 +699,25 @@ __global__ void __launch_bounds__(320, 1)
                     if (has_tiles) {
                         if (qseg > 0) ok = ok && spin_phase<false>(bar(BR::QEMPTY), (qseg - 1) & 1, wc, status);
                         {
-                            const int n = tid >> 4, part = tid & 15;  // 16 threads per column, 36 values each
+                            // TPC threads per column (16 or 8), each 2 * WPT of the 576 values
+                            constexpr int TPC = NSM / NG, WPT = kDqk / 2 / TPC;
+                            const int n = tid / TPC, part = tid % TPC;
                             const int ng = grp * NG + n;
                             float amax = 0.f;
                             if (ng < p.ncols) {
                                 const uint32_t *qw =
                                     reinterpret_cast<const uint32_t *>(p.q + ((int64_t)b * p.ncols + ng) * kDqk) +
-                                    18 * part;
+                                    WPT * part;
 #pragma unroll 6
-                                for (int i = 0; i < 18; ++i) {
+                                for (int i = 0; i < WPT; ++i) {
                                     const uint32_t w2 = __ldg(qw + i);
                                     amax = fmaxf(amax, fmaxf(fabsf(__uint_as_float(w2 << 16)),
                                                              fabsf(__uint_as_float(w2 & 0xFFFF0000u))));
                                 }
                             }
 #pragma unroll
-                            for (int o = 8; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                            for (int o = TPC / 2; o >= 1; o >>= 1)
+                                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                             int c = 0;
                             if (amax > 0.f && amax < INFINITY) {
                                 // c = 8 - ceil(log2 amax), read off the fp32 exponent and mantissa fields
@@ -756,7 +772,7 @@ __global__ void __launch_bounds__(320, 1)
                         ++qseg;
                     }
 #pragma unroll
-                    for (int n = 0; n < NH; ++n) qv[n] = qsc[NG + 8 * half + n];
+                    for (int n = 0; n < NH; ++n) qv[n] = qsc[NG + 16 * (n >> 3) + 8 * half + (n & 7)];
                 } else {
 #pragma unroll
                     for (int n = 0; n < NH; ++n) qv[n] = 1.f;
@@ -792,7 +808,23 @@ __global__ void __launch_bounds__(320, 1)
                         qlen_b == p.q_len && (t + 1) * kTileRows <= (p.causal ? L - qlen_b + 1 : L);
                     bool waited_prev = false, rescale_any = false, sent_next = false;
                     float xc[C::CH][8];  // CH > 1: full scores of this thread's columns, in registers
-                    if constexpr (C::CH > 1) {
+                    if constexpr (C::KV8) {
+                        // scores against Q_hi and against Q_lo, added; each CTA holds whole rows (no exchange)
+                        float xl[C::CH][8];
+#pragma unroll
+                        for (int ch = 0; ch < C::CH; ++ch) {
+                            tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * C::NS + 16 * ch + 8 * half, xc[ch]);
+                            tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * C::NS + NG + 16 * ch + 8 * half, xl[ch]);
+                        }
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int ch = 0; ch < C::CH; ++ch)
+#pragma unroll
+                            for (int n = 0; n < 8; ++n) xc[ch][n] += xl[ch][n];
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(BR::SEMPTY + (k & 1)));
+                    } else if constexpr (C::CH > 1) {
                         // (a) add the peer's partial S^T of tile k to ours in registers; free the TMEM
                         //     buffer and the peer's slots; (b) send our partial of tile k+1 so it travels
                         //     while tile k's softmax runs.
@@ -832,18 +864,9 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                     for (int ch = 0; ch < C::CH; ++ch) {
                         float(&x)[8] = xc[ch];
-                        if constexpr (C::CH == 1) {
+                        if constexpr (C::CH == 1 && !C::KV8) {
                             tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * C::NS + 8 * half, x);
-                            if constexpr (C::KV8) {
-                                // scores against Q_hi and against Q_lo, added
-                                float xl[8];
-                                tmem_ld8(tmem + lane_addr + C::S_COL + (k & 1) * C::NS + NG + 8 * half, xl);
-                                tmem_wait_ld();
-#pragma unroll
-                                for (int n = 0; n < 8; ++n) x[n] += xl[n];
-                            } else {
-                                tmem_wait_ld();
-                            }
+                            tmem_wait_ld();
                             tc_fence_before();
                             __syncwarp();
                             if (lane == 0) mbar_arrive(bar(BR::SEMPTY + (k & 1)));
@@ -1047,7 +1070,7 @@ __global__ void __launch_bounds__(320, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(BR::PFULL + pb));
                     }
-                    if constexpr (C::CH > 1) {
+                    if constexpr (C::CH > 1 && !C::KV8) {
                         if (k + 1 < k_total && !sent_next) send_tile(k + 1);
                     }
                 }
@@ -1101,97 +1124,96 @@ __global__ void __launch_bounds__(320, 1)
                     // ---- merge of the two CTAs' partials of this segment (disjoint tiles, all 512 latent rows
                     //      each): send the peer the two M-tiles it writes and this CTA's (m, l) of these columns,
                     //      receive the same, and combine by the log-sum-exp rule.
-                    float ms[8], ls[8], ov[4][8];
+                    float ms[NH], ls[NH], own[2][NH];
 #pragma unroll
-                    for (int n = 0; n < 8; ++n) {
-                        const int cn = 8 * half + n;
+                    for (int n = 0; n < NH; ++n) {
+                        const int cn = 16 * (n >> 3) + 8 * half + (n & 7);
                         ls[n] = redl[cn] + redl[NG + cn] + redl[2 * NG + cn] + redl[3 * NG + cn];
                         ms[n] = has_tiles ? m[n] : -INFINITY;
                     }
+                    const uint32_t x_peer = map_to_rank(sbase + C::OFF_XM, peer);
+                    const uint32_t xml = 2u * C::XM_TILE + (uint32_t)sw * (2u * NH * 4u);
+                    // This CTA's merge area (its Q and P^T buffers) is idle now: every thread has passed
+                    // the barrier after the segment's last step 3, whose completion it waited for, and
+                    // the score MMAs completed before their last S^T was read.  Tell the peer's warp,
+                    // then wait until the peer says the same of its area.
+                    if (lane == 0) mbar_arrive_remote(xfree_remote);
+                    ok = ok && spin_phase<true>(bar(BR::XFREE + sw), mseg & 1, wc, status);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        float hi[8], lo[8];
-                        if (has_tiles) {
-                            tmem_ld8(tmem + lane_addr + C::O_COL + i * C::NP + 8 * half, hi);
-                            tmem_ld8(tmem + lane_addr + C::O_COL + i * C::NP + NG + 8 * half, lo);
-                            tmem_wait_ld();
+                    for (int ch = 0; ch < C::CH; ++ch) {
+                        // O^T of the 4 M-tiles for this thread's row and 8 columns (hi + lo)
+                        const uint32_t xcol = (uint32_t)row * C::XM_ROW + (uint32_t)(16 * ch + 8 * half) * 4u;
+#pragma unroll
+                        for (int mt = 0; mt < 4; ++mt) {
+                            float hi[8], lo[8];
+                            if (has_tiles) {
+                                tmem_ld8(tmem + lane_addr + C::O_COL + mt * C::NP + 16 * ch + 8 * half, hi);
+                                tmem_ld8(tmem + lane_addr + C::O_COL + mt * C::NP + NG + 16 * ch + 8 * half, lo);
+                                tmem_wait_ld();
+                            }
+                            float v[8];
+#pragma unroll
+                            for (int n = 0; n < 8; ++n) v[n] = has_tiles ? hi[n] + lo[n] : 0.f;
+                            // M-tiles 2 rank, 2 rank + 1 stay here, the other two go to the peer (selects,
+                            // so that nothing is indexed by the rank at run time)
+                            const bool mine = (mt >> 1) == (int)rank;
+                            if (mine) {
+#pragma unroll
+                                for (int n = 0; n < 8; ++n) own[mt & 1][8 * ch + n] = v[n];
+                            } else if (ok) {
+                                const uint32_t dst = x_peer + (uint32_t)(mt & 1) * C::XM_TILE + xcol;
+                                st_async_v4(dst, __float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                                            __float_as_uint(v[3]), xfull_remote);
+                                st_async_v4(dst + 16u, __float_as_uint(v[4]), __float_as_uint(v[5]),
+                                            __float_as_uint(v[6]), __float_as_uint(v[7]), xfull_remote);
+                            }
                         }
-#pragma unroll
-                        for (int n = 0; n < 8; ++n) ov[i][n] = has_tiles ? hi[n] + lo[n] : 0.f;
                     }
                     tc_fence_before();
-                    // M-tiles 2 rank, 2 rank + 1 stay here, the other two go to the peer (selects, so that
-                    // nothing is indexed by the rank at run time)
-                    float own[2][8], oth[2][8];
+                    if (ok && lane == 0) {
 #pragma unroll
-                    for (int j = 0; j < 2; ++j)
-#pragma unroll
-                        for (int n = 0; n < 8; ++n) {
-                            own[j][n] = rank == 0 ? ov[j][n] : ov[2 + j][n];
-                            oth[j][n] = rank == 0 ? ov[2 + j][n] : ov[j][n];
-                        }
-                    const uint32_t x_peer = map_to_rank(sbase + C::OFF_X, peer);
-                    const uint32_t xrow = (uint32_t)row * 64u + (uint32_t)half * 32u;
-                    const uint32_t xml = 2u * 8192u + (uint32_t)sw * 64u;
-                    ok = ok && spin_phase<true>(bar(BR::XFREE + sw), (mseg & 1) ^ 1, wc, status);
-                    if (ok) {
-#pragma unroll
-                        for (int j = 0; j < 2; ++j) {
-                            const float *v = oth[j];
-                            st_async_v4(x_peer + 8192u * j + xrow, __float_as_uint(v[0]), __float_as_uint(v[1]),
-                                        __float_as_uint(v[2]), __float_as_uint(v[3]), xfull_remote);
-                            st_async_v4(x_peer + 8192u * j + xrow + 16u, __float_as_uint(v[4]), __float_as_uint(v[5]),
-                                        __float_as_uint(v[6]), __float_as_uint(v[7]), xfull_remote);
-                        }
-                        if (lane == 0) {
-                            st_async_v4(x_peer + xml, __float_as_uint(ms[0]), __float_as_uint(ms[1]),
-                                        __float_as_uint(ms[2]), __float_as_uint(ms[3]), xfull_remote);
-                            st_async_v4(x_peer + xml + 16u, __float_as_uint(ms[4]), __float_as_uint(ms[5]),
-                                        __float_as_uint(ms[6]), __float_as_uint(ms[7]), xfull_remote);
-                            st_async_v4(x_peer + xml + 32u, __float_as_uint(ls[0]), __float_as_uint(ls[1]),
-                                        __float_as_uint(ls[2]), __float_as_uint(ls[3]), xfull_remote);
-                            st_async_v4(x_peer + xml + 48u, __float_as_uint(ls[4]), __float_as_uint(ls[5]),
-                                        __float_as_uint(ls[6]), __float_as_uint(ls[7]), xfull_remote);
+                        for (int n4 = 0; n4 < NH; n4 += 4) {
+                            st_async_v4(x_peer + xml + 4u * n4, __float_as_uint(ms[n4]), __float_as_uint(ms[n4 + 1]),
+                                        __float_as_uint(ms[n4 + 2]), __float_as_uint(ms[n4 + 3]), xfull_remote);
+                            st_async_v4(x_peer + xml + 4u * (NH + n4), __float_as_uint(ls[n4]),
+                                        __float_as_uint(ls[n4 + 1]), __float_as_uint(ls[n4 + 2]),
+                                        __float_as_uint(ls[n4 + 3]), xfull_remote);
                         }
                     }
-                    if (lane == 0) mbar_arrive_expect_tx(bar(BR::XFULL + sw), 32 * 64 + 64);
+                    if (lane == 0) mbar_arrive_expect_tx(bar(BR::XFULL + sw), 32 * 2 * NH * 4 + 2 * NH * 4);
                     ok = ok && spin_phase<true>(bar(BR::XFULL + sw), mseg & 1, wc, status);
                     ++mseg;
-                    float op[2][8], mp[8], lp[8];
-                    {
-                        const float *xs = reinterpret_cast<const float *>(smem + C::OFF_X);
-#pragma unroll
-                        for (int j = 0; j < 2; ++j)
-#pragma unroll
-                            for (int n = 0; n < 8; ++n) op[j][n] = xs[(8192u * j + xrow) / 4 + n];
-#pragma unroll
-                        for (int n = 0; n < 8; ++n) {
-                            mp[n] = xs[xml / 4 + n];
-                            lp[n] = xs[xml / 4 + 8 + n];
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_remote(xfree_remote);
+                    // (the area is written again only by the next segment's Q quantisation, after a
+                    // barrier of all softmax warps, i.e. after every warp has read its part)
                     if (!named_bar_and(SMX, NSM, ok)) {
                         stop = true;
                         break;
                     }
-                    float lse_n[8];
+                    const float *xs = reinterpret_cast<const float *>(smem + C::OFF_XM);
 #pragma unroll
-                    for (int n = 0; n < 8; ++n) {
-                        const float mm = fmaxf(ms[n], mp[n]);
-                        const float as = ms[n] == -INFINITY ? 0.f : fast_exp2(ms[n] - mm);
-                        const float ap = mp[n] == -INFINITY ? 0.f : fast_exp2(mp[n] - mm);
-                        const float l = ls[n] * as + lp[n] * ap;
-                        const bool empty = !(l > 0.f) || mm == -INFINITY;
-                        // the stored p carried a factor 2^4
-                        const float inv = empty ? 0.f : 0.0625f / l;
-                        lse_n[n] = empty ? -INFINITY : (mm + __log2f(l)) * 0.69314718055994531f;
+                    for (int ch = 0; ch < C::CH; ++ch) {
+                        const uint32_t xcol = (uint32_t)row * C::XM_ROW + (uint32_t)(16 * ch + 8 * half) * 4u;
+                        float lse_n[8];
 #pragma unroll
-                        for (int j = 0; j < 2; ++j)
-                            store_o(0, j, n, (own[j][n] * as + op[j][n] * ap) * inv);
+                        for (int n = 0; n < 8; ++n) {
+                            const int li = 8 * ch + n;
+                            const float mp = xs[xml / 4 + li], lp = xs[xml / 4 + NH + li];
+                            const float mm = fmaxf(ms[li], mp);
+                            const float as = ms[li] == -INFINITY ? 0.f : fast_exp2(ms[li] - mm);
+                            const float ap = mp == -INFINITY ? 0.f : fast_exp2(mp - mm);
+                            const float l = ls[li] * as + lp * ap;
+                            const bool empty = !(l > 0.f) || mm == -INFINITY;
+                            // the stored p carried a factor 2^4
+                            const float inv = empty ? 0.f : 0.0625f / l;
+                            lse_n[n] = empty ? -INFINITY : (mm + __log2f(l)) * 0.69314718055994531f;
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                const float op = xs[(j * C::XM_TILE + xcol) / 4 + n];
+                                store_o(ch, j, n, (own[j][li] * as + op * ap) * inv);
+                            }
+                        }
+                        store_lse(ch, lse_n);
                     }
-                    store_lse(0, lse_n);
                 } else {
 #pragma unroll
                 for (int ch = 0; ch < C::CH; ++ch) {
@@ -1242,7 +1264,7 @@ __global__ void __launch_bounds__(320, 1)
                         const int d4 = 256 * (int)rank + 4 * (tid & 63), nq0 = (tid >> 6) * NQ;
                         const int nn = p.ncols - grp * NG < NG ? p.ncols - grp * NG : NG;
                         const float *op = p.opart + ((int64_t)s0 * p.ncols + grp * NG + nq0) * kDv + d4;
-                        float *ls = reinterpret_cast<float *>(smem + C::OFF_P);  // [nsplit][NG]
+                        float *ls = reinterpret_cast<float *>(smem + C::OFF_STAGE);  // [nsplit][NG]
                         float *lt = ls + nsplit * NG;                             // [NG]
                         float4 v[U][NQ];
                         auto load_batch = [&](int sp0) {

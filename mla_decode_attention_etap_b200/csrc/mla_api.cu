@@ -102,6 +102,9 @@ int ensure_smem_attr() {
         e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg16E4>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::PairCfg16E4::SMEM_ALLOC);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg32E4>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::PairCfg32E4::SMEM_ALLOC);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         done[dev] = true;
     }
     return MLA_OK;
@@ -260,7 +263,6 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
     const bool fp8 = kv_scale != nullptr;
     int st = check_shape(batch, q_len, num_heads, num_sms);
     if (st != MLA_OK) return st;
-    if (fp8 && q_len * num_heads > 16) return MLA_ERR_UNSUPPORTED;
     if (!q || !kv || !seqlens || !o || !lse || !workspace) return MLA_ERR_INVALID_ARG;
     if (!(softmax_scale > 0.f) || !std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return MLA_ERR_INVALID_ARG;
@@ -337,17 +339,20 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
     p.counters = reinterpret_cast<int32_t *>(ws + lay.counters);
     p.slots = lay.slots;
     // splits of a sequence are at most the work units (CTA pairs per column group)
-    const int max_splits = fp8        ? mla::PairCfg16E4::MERGE_MAX_SPLITS
-                           : ng == 16 ? mla::PairCfg16::MERGE_MAX_SPLITS
-                                      : mla::PairCfg32::MERGE_MAX_SPLITS;
+    const int max_splits = fp8 ? (ng == 16 ? mla::PairCfg16E4::MERGE_MAX_SPLITS : mla::PairCfg32E4::MERGE_MAX_SPLITS)
+                               : (ng == 16 ? mla::PairCfg16::MERGE_MAX_SPLITS : mla::PairCfg32::MERGE_MAX_SPLITS);
     const bool separate_combine = !(flags & MLA_FLAG_SKIP_COMBINE) && lay.ctas > max_splits;
     p.fuse_merge = ((flags & MLA_FLAG_SKIP_COMBINE) || separate_combine) ? 0 : 1;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int clusters = lay.ctas * lay.groups;
-    cudaError_t e = fp8        ? launch_pair<mla::PairCfg16E4>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s)
-                    : ng == 16 ? launch_pair<mla::PairCfg16>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s)
-                               : launch_pair<mla::PairCfg32>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s);
+    cudaError_t e;
+    if (fp8)
+        e = ng == 16 ? launch_pair<mla::PairCfg16E4>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s)
+                     : launch_pair<mla::PairCfg32E4>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s);
+    else
+        e = ng == 16 ? launch_pair<mla::PairCfg16>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s)
+                     : launch_pair<mla::PairCfg32>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s);
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");

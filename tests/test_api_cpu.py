@@ -119,7 +119,7 @@ def fwd_fp8(**kw):
 @pytest.mark.parametrize("kw,code", [
     (dict(kv_scale=0), -1),                     # the FP8 entry needs its row scales
     (dict(kv8=0), -1),
-    (dict(num_heads=32), -2), (dict(q_len=2), -2),   # more than 16 query columns
+    (dict(num_heads=2048), -2),                 # more than MLA_MAX_COLUMNS query columns
     (dict(scale=0.0), -1), (dict(causal=3), -1),
     (dict(kv8=A + 8), -3), (dict(kv_scale=A + 2), -3), (dict(q_lens=A + 2), -3),
     (dict(ws_bytes=100), -4),

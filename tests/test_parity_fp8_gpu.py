@@ -162,15 +162,39 @@ def test_full_size_64k_sampled_sequences():
     assert_parity(o[idx], lse[idx], o_ref, lse_ref, what="fp8 64K sampled")
 
 
-def test_unsupported_column_count_is_rejected():
-    w = fp8(1, 32, [100], seed=110)
-    dev = torch.device("cuda")
-    dec = MlaDecoder(1, 1, 32, device=dev)
-    sl = w.seqlens.to(dev)
-    dec.plan(sl)
-    with pytest.raises(MlaError) as ei:
-        dec.fwd_fp8(w.q.to(dev), w.kv8.to(dev), w.kv_scale.to(dev), sl)
-    assert ei.value.code == -2
+@pytest.mark.parametrize("heads,q_len,causal,lens", [
+    (32, 1, False, [3000, 257, 1]),          # one group of 32 columns
+    (16, 4, True, [2100, 3, 700]),           # two groups (the speculative-verify shape)
+    (128, 1, False, [1100, 300]),            # four groups
+    (16, 16, True, [1500, 16, 17]),          # append: eight groups
+    (20, 1, False, [999, 4097]),             # a partly empty last group
+])
+def test_column_groups_of_32(heads, q_len, causal, lens):
+    w = _poison(fp8(len(lens), heads, lens, q_len=q_len, causal=causal, seed=120 + heads + q_len,
+                    l_max=max(lens) + 40, spike_frac=0.05 if causal else 0.0))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"fp8 h={heads} q={q_len}")
+
+
+def test_column_groups_of_32_ragged_paged():
+    lens = [900, 3, 1300, 257]
+    q_lens = [4, 0, 1, 3]
+    w = _poison(fp8(len(lens), 16, lens, q_len=4, causal=True, paged=True, seed=130, q_lens=q_lens,
+                    extra_blocks=3))
+    o, lse, st, _ = run_cuda(w)
+    assert st == 0
+    for b, qb in enumerate(q_lens):
+        assert np.all(o[b, qb:] == 0) and np.all(np.isneginf(lse[b, qb:]))
+    assert_parity(o, lse, *run_oracle(w), what="fp8 ragged paged")
+
+
+@pytest.mark.parametrize("n_sms", [2, 148, 1024])
+def test_column_groups_of_32_split_counts(n_sms):
+    w = fp8(3, 16, [5000, 700, 2100], q_len=2, causal=True, seed=131)
+    o, lse, st, _ = run_cuda(w, n_sms=n_sms)
+    assert st == 0
+    assert_parity(o, lse, *run_oracle(w), what=f"fp8 q2 n_sms={n_sms}")
 
 
 def test_bounded_waits_report_timeout_and_context_survives():
