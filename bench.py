@@ -70,6 +70,7 @@ WORKLOADS = {
     "b64_h16_paged_fp8": dict(kind="b64_paged_fp8"),
     "b16_h16_q4_causal_fp8": dict(kind="q4_causal_fp8"),
     "b32_h128_paged_fp8": dict(kind="b32_h128_fp8"),
+    "b16_h16_append_q16_fp8": dict(kind="append_q16_fp8"),
 }
 
 
@@ -130,6 +131,10 @@ def make_workload(name: str, rank: int, device):
         lens = W.draw_seqlens(32, 8192, 32768, seed)
         return (W.make_workload(32, 128, lens, paged=True, seed=seed, device=device, kv_dtype="e4m3"),
                 "mla_decode_b32_h128_q1_Lunif8192to32768_paged64_e4m3cache")
+    if kind == "append_q16_fp8":
+        return (W.make_workload(16, 16, [32768] * 16, q_len=16, causal=True, seed=seed, device=device,
+                                kv_dtype="e4m3"),
+                "mla_decode_b16_h16_append_q16_causal_L32768_e4m3cache")
     if kind == "b64_paged_fp8":
         return (W.workload_b64_h16_paged_fp8(seed=seed, device=device),
                 "mla_decode_b64_h16_q1_Lunif1to65536_paged64_e4m3cache")
