@@ -1257,7 +1257,8 @@ __global__ void __launch_bounds__(320, 1)
                     if (*merge_flag) {
                         // thread = 4 consecutive latent rows (one float4) x NG/4 columns.  The first
                         // U splits' partial outputs are in flight while the LSE partials are staged in
-                        // the idle P^T buffers (the last step 3 has completed) and merged per column.
+                        // an idle buffer (bf16: the P^T buffers, whose last step 3 has completed; E4M3:
+                        // the Q area, read by no MMA before the next segment) and merged per column.
                         constexpr int NQ = NG / 4, U = 16 / NQ;
                         const int s0 = seq_info[4 * b + 3];
                         const int tid = (warp - 2) * 32 + lane;
@@ -1316,7 +1317,8 @@ __global__ void __launch_bounds__(320, 1)
                             *reinterpret_cast<uint2 *>(p.o + ((int64_t)b * p.ncols + grp * NG + nq0 + j) * kDv + d4) = packed;
                             if (rank == 0 && (tid & 63) == 0) p.lse[(int64_t)b * p.ncols + grp * NG + nq0 + j] = lt[nq0 + j];
                         }
-                        // ls/lt are next overwritten as P^T after the next tile's vote barrier
+                        // ls/lt are next overwritten after a barrier of all softmax warps: as P^T (bf16)
+                        // or by the next segment's Q quantisation (E4M3)
                         if (row == 0 && half == 0) *cnt = 0;  // ready for the next call
                     }
                 }
