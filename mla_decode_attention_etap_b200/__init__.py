@@ -96,6 +96,55 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _require(t, name: str, dtype, device, min_numel: int = 0, dim: Optional[int] = None,
+             last: Optional[int] = None, min_rows: int = 0) -> None:
+    """Reject a tensor whose raw pointer the library could not use safely: the C ABI sees only the
+    pointer, so dtype, device, layout and size are checked here (TypeError / ValueError)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device} (all tensors on the device of q)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name}: {t.dim()}-D, expected {dim}-D")
+    if last is not None and (t.dim() == 0 or t.shape[-1] != last):
+        raise ValueError(f"{name}: last dimension must be {last}, got shape {tuple(t.shape)}")
+    if min_rows and (t.dim() == 0 or t.shape[0] < min_rows):
+        raise ValueError(f"{name}: needs at least {min_rows} rows in dimension 0, got shape {tuple(t.shape)}")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name}: {t.numel()} elements, needs at least {min_numel}")
+
+
+def check_decode_args(q, kv, seqlens, block_table, o, lse, workspace, q_lens=None, kv_scale=None) -> None:
+    """Shapes, dtypes and devices of a decode call (``kv_scale`` given: the FP8 cache, ``kv`` uint8)."""
+    if not isinstance(q, torch.Tensor):
+        raise TypeError("q: expected a torch.Tensor")
+    dev = q.device
+    _require(q, "q", torch.bfloat16, dev, dim=4, last=D_QK)
+    B, q_len, h, _ = q.shape
+    fp8 = kv_scale is not None
+    _require(kv, "kv8" if fp8 else "kv", torch.uint8 if fp8 else torch.bfloat16, dev, dim=3, last=D_QK,
+             min_rows=0 if block_table is not None else B)
+    _require(seqlens, "seqlens", torch.int32, dev, min_numel=B, dim=1)
+    if block_table is not None:
+        _require(block_table, "block_table", torch.int32, dev, dim=2, min_rows=B)
+    if q_lens is not None:
+        _require(q_lens, "q_lens", torch.int32, dev, min_numel=B, dim=1)
+    if fp8:
+        _require(kv_scale, "kv_scale", torch.float32, dev, min_numel=kv.shape[0] * kv.shape[1])
+    _require(o, "o", torch.bfloat16, dev, min_numel=B * q_len * h * D_V)
+    _require(lse, "lse", torch.float32, dev, min_numel=B * q_len * h)
+    _require(workspace, "workspace", None, dev)
+
+
+def _require_cuda(t, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor")
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
@@ -115,6 +164,9 @@ def mla_decode_workspace_size(batch: int, q_len: int, num_heads: int, n_sms: int
 
 def mla_decode_plan(seqlens: torch.Tensor, q_len: int, num_heads: int, workspace: torch.Tensor, n_sms: int,
                     stream=None) -> None:
+    _require_cuda(seqlens, "seqlens")
+    _require(seqlens, "seqlens", torch.int32, seqlens.device, dim=1)
+    _require(workspace, "workspace", None, seqlens.device)
     _check(lib().mla_decode_plan(_ptr(seqlens), seqlens.numel(), q_len, num_heads, n_sms, _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)), "mla_decode_plan")
 
@@ -123,6 +175,8 @@ def mla_decode_fwd(q, kv, seqlens, block_table, softmax_scale, causal, o, lse, w
                    stream=None, q_lens=None) -> None:
     """``q_lens`` (optional int32 device tensor [B]): ragged batch, q_lens[b] real query tokens of the
     q_len rows of sequence b (``mla_decode_fwd_ragged``)."""
+    _require_cuda(q, "q")
+    check_decode_args(q, kv, seqlens, block_table, o, lse, workspace, q_lens)
     B, q_len, h, _ = q.shape
     if block_table is not None:
         kv_rows, max_blocks = kv.shape[0] * kv.shape[1], block_table.shape[1]
@@ -144,13 +198,14 @@ def mla_decode_fwd(q, kv, seqlens, block_table, softmax_scale, causal, o, lse, w
 def mla_decode_fwd_fp8(q, kv8, kv_scale, seqlens, block_table, softmax_scale, causal, o, lse, workspace, n_sms,
                        flags=0, stream=None, q_lens=None) -> None:
     """Decode over an FP8 cache: ``kv8`` uint8 E4M3 codes laid out like the bf16 cache, ``kv_scale``
-    fp32 with one scale per cache row (``mla_decode_fwd_fp8``; h * q_len <= 16)."""
+    fp32 with one scale per cache row (``mla_decode_fwd_fp8``; up to MLA_MAX_COLUMNS query columns)."""
+    _require_cuda(q, "q")
+    check_decode_args(q, kv8, seqlens, block_table, o, lse, workspace, q_lens, kv_scale=kv_scale)
     B, q_len, h, _ = q.shape
     if block_table is not None:
         kv_rows, max_blocks = kv8.shape[0] * kv8.shape[1], block_table.shape[1]
     else:
         kv_rows, max_blocks = kv8.shape[1], 0
-    assert kv8.dtype == torch.uint8 and kv_scale.dtype == torch.float32
     _check(lib().mla_decode_fwd_fp8(_ptr(q), _ptr(kv8), _ptr(kv_scale), _ptr(seqlens), _ptr(q_lens),
                                     _ptr(block_table), B, q_len, h, kv_rows, max_blocks, float(softmax_scale),
                                     int(bool(causal)), _ptr(o), _ptr(lse), _ptr(workspace),
@@ -161,6 +216,9 @@ def mla_decode_fwd_fp8(q, kv8, kv_scale, seqlens, block_table, softmax_scale, ca
 def mla_stream_probe(kv, units: int, err, stream=None) -> None:
     """Stream ``kv`` ([..., 576] bf16, rows a multiple of 128) with the decode's TMA read pattern and
     no computation (a bandwidth probe).  ``err``: int32 device tensor [1], zeroed by the caller."""
+    _require_cuda(kv, "kv")
+    _require(kv, "kv", torch.bfloat16, kv.device, last=D_QK)
+    _require(err, "err", torch.int32, kv.device, min_numel=1)
     rows = kv.numel() // 576
     _check(lib().mla_stream_probe(_ptr(kv), rows, units, _ptr(err), _stream(stream)), "mla_stream_probe")
 
@@ -168,16 +226,24 @@ def mla_stream_probe(kv, units: int, err, stream=None) -> None:
 def mla_form_ablation(form: int, heads: int, streams: int, tiles: int, cycles, err, stream=None) -> None:
     """Tensor-core instructions of ``tiles`` KV tiles per CTA in the transposed (form 0) or untransposed
     (form 1) layout; ``cycles``: uint64-compatible int64 device tensor [ctas], ``err``: int32 [1] zeroed."""
+    _require_cuda(cycles, "cycles")
+    _require(cycles, "cycles", torch.int64, cycles.device, min_numel=1)
+    _require(err, "err", torch.int32, cycles.device, min_numel=1)
     _check(lib().mla_form_ablation(form, heads, streams, tiles, cycles.numel(), _ptr(cycles), _ptr(err),
                                    _stream(stream)), "mla_form_ablation")
 
 
 def mla_combine(workspace, batch, q_len, num_heads, n_sms, o, lse, stream=None) -> None:
+    _require_cuda(o, "o")
+    _require(o, "o", torch.bfloat16, o.device, min_numel=batch * q_len * num_heads * D_V)
+    _require(lse, "lse", torch.float32, o.device, min_numel=batch * q_len * num_heads)
+    _require(workspace, "workspace", None, o.device)
     _check(lib().mla_combine(_ptr(workspace), batch, q_len, num_heads, n_sms, _ptr(o), _ptr(lse), _stream(stream)),
            "mla_combine")
 
 
 def mla_decode_read_status(workspace, stream=None) -> int:
+    _require_cuda(workspace, "workspace")
     out = ctypes.c_int(0)
     _check(lib().mla_decode_read_status(_ptr(workspace), ctypes.byref(out), _stream(stream)),
            "mla_decode_read_status")

@@ -9,6 +9,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import mla_decode_attention_etap_b200 as m
 
@@ -146,3 +147,89 @@ def test_measurement_helpers_reject():
     assert L.mla_stream_probe(vp(A), 100, 74, vp(A), None) == -1      # rows not a multiple of 128
     assert L.mla_stream_probe(vp(A), 256, 0, vp(A), None) == -1
     assert L.mla_stream_probe(vp(A + 8), 256, 74, vp(A), None) == -3
+
+
+# ---------------------------------------------------------------------------- binding-level guards
+def _decode_args(B=2, q_len=1, h=16, rows=130, paged=False, fp8=False):
+    kv_shape = (3, 64, 576) if paged else (B, rows, 576)
+    a = dict(q=torch.zeros(B, q_len, h, 576, dtype=torch.bfloat16),
+             kv=torch.zeros(kv_shape, dtype=torch.uint8 if fp8 else torch.bfloat16),
+             seqlens=torch.zeros(B, dtype=torch.int32),
+             block_table=torch.zeros(B, 3, dtype=torch.int32) if paged else None,
+             o=torch.zeros(B, q_len, h, 512, dtype=torch.bfloat16),
+             lse=torch.zeros(B, q_len, h, dtype=torch.float32),
+             workspace=torch.zeros(1024, dtype=torch.uint8),
+             q_lens=None,
+             kv_scale=torch.ones(kv_shape[:2], dtype=torch.float32) if fp8 else None)
+    return a
+
+
+@pytest.mark.parametrize("paged,fp8", [(False, False), (True, False), (False, True), (True, True)])
+def test_decode_guards_accept_well_formed_arguments(paged, fp8):
+    m.check_decode_args(**_decode_args(paged=paged, fp8=fp8))
+
+
+BAD = [
+    ("q", lambda a: a["q"].float(), TypeError),
+    ("q", lambda a: a["q"][..., :512].contiguous(), ValueError),
+    ("q", lambda a: torch.zeros(2, 1, 16, 1152, dtype=torch.bfloat16)[..., ::2], ValueError),  # strided view
+    ("kv", lambda a: a["kv"][:1], ValueError),              # fewer cache rows than sequences
+    ("kv", lambda a: a["kv"].to(torch.float16), TypeError),
+    ("seqlens", lambda a: a["seqlens"].long(), TypeError),
+    ("seqlens", lambda a: a["seqlens"][:1], ValueError),
+    ("o", lambda a: a["o"][:, :, :, :256].contiguous(), ValueError),
+    ("o", lambda a: a["o"].float(), TypeError),
+    ("lse", lambda a: a["lse"][:1], ValueError),
+    ("q_lens", lambda a: torch.zeros(1, dtype=torch.int32), ValueError),
+    ("workspace", lambda a: a["workspace"][::2], ValueError),
+]
+
+
+@pytest.mark.parametrize("name,make,exc", BAD)
+def test_decode_guards_reject(name, make, exc):
+    a = _decode_args()
+    a[name] = make(a)
+    with pytest.raises(exc):
+        m.check_decode_args(**a)
+
+
+def test_decode_guards_reject_paged_and_fp8_mistakes():
+    a = _decode_args(paged=True)
+    a["block_table"] = a["block_table"][:1]
+    with pytest.raises(ValueError):
+        m.check_decode_args(**a)
+    a = _decode_args(fp8=True)
+    a["kv_scale"] = a["kv_scale"][:1]
+    with pytest.raises(ValueError):
+        m.check_decode_args(**a)
+    a = _decode_args(fp8=True)
+    a["kv"] = a["kv"].to(torch.bfloat16)
+    with pytest.raises(TypeError):
+        m.check_decode_args(**a)
+
+
+def test_wrappers_refuse_host_tensors_before_any_launch():
+    a = _decode_args()
+    with pytest.raises(ValueError, match="CUDA"):
+        m.mla_decode_fwd(a["q"], a["kv"], a["seqlens"], None, 0.04, False, a["o"], a["lse"], a["workspace"], 148)
+    with pytest.raises(ValueError, match="CUDA"):
+        m.mla_decode_plan(a["seqlens"], 1, 16, a["workspace"], 148)
+    with pytest.raises(ValueError, match="CUDA"):
+        m.mla_combine(a["workspace"], 2, 1, 16, 148, a["o"], a["lse"])
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(paged=True), dict(kv_dtype="e4m3"), dict(paged=True, kv_dtype="e4m3"),
+                                dict(q_len=4, causal=True, q_lens=[4, 1, 3]), dict(num_heads=128, paged=True)])
+def test_decode_guards_accept_what_the_parity_tests_pass(kw):
+    """The arguments tests/parity.py builds for the GPU (here on the host) pass the binding's guards."""
+    from mla_decode_attention_etap_b200 import workloads as W
+    kw = dict(kw)
+    heads = kw.pop("num_heads", 16)
+    w = W.make_workload(3, heads, [700, 5, 130], seed=3, **kw)
+    o = torch.full((w.batch, w.q_len, w.num_heads, 512), float("nan"), dtype=torch.bfloat16)
+    lse = torch.full((w.batch, w.q_len, w.num_heads), float("nan"), dtype=torch.float32)
+    ws = torch.empty(4096, dtype=torch.uint8)
+    if w.fp8:
+        m.check_decode_args(w.q, w.kv8, w.seqlens, w.block_table, o, lse, ws, w.q_lens, kv_scale=w.kv_scale)
+    else:
+        m.check_decode_args(w.q, w.kv, w.seqlens, w.block_table, o, lse, ws, w.q_lens)
