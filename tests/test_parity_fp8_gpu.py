@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 import torch
 
-from mla_decode_attention_etap_b200 import MlaDecoder, MlaError
+from mla_decode_attention_etap_b200 import MlaDecoder
 from mla_decode_attention_etap_b200 import workloads as W
 from tests.parity import assert_parity, run_cuda, run_oracle
 
