@@ -1,4 +1,5 @@
-"""Host-side pieces of bench.py: the kernel-source hash that keys the profiled DRAM traffic."""
+"""Host-side pieces of bench.py: the kernel-source hash that keys the profiled DRAM traffic, and the
+roofline peaks (measured file, else the recipe fallback)."""
 
 import bench
 
@@ -15,3 +16,17 @@ def test_profiled_traffic_matches_the_current_kernel_source():
     assert t is not None
     # read traffic within a few percent of the algorithmic KV bytes of the launch
     assert 1.0 <= t / (16 * 65536 * 1152) < 1.05
+
+
+def test_peaks_come_from_the_measured_file_else_the_recipe_fallback(monkeypatch, tmp_path):
+    import json
+    import os
+    if os.path.exists(bench.PEAKS_FILE):
+        with open(bench.PEAKS_FILE) as f:
+            pk = json.load(f)
+        hbm, tc, tcs, src = bench.load_peaks()
+        assert src == "measured"
+        assert (hbm, tc, tcs) == (pk["hbm_gbs"], pk["bf16_tflops"], pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    # the profiling recipe's fallback: 6.65 TB/s and 1.59 PFLOP/s (burst), about 1.4 sustained
+    monkeypatch.setattr(bench, "PEAKS_FILE", str(tmp_path / "absent.json"))
+    assert bench.load_peaks() == (6650.0, 1590.0, 1400.0, "fallback")
