@@ -132,7 +132,7 @@ MLA_API int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens
 /*
  * Ragged multi-token decode: as mla_decode_fwd, with a different number of new
  * query tokens per sequence.  The pages decode one token per forward and name
- * more as a limitation (FlashMLA-ETAP technical summary, "Discussion"); this is
+ * more as a limitation (FlashMLA-ETAP Chinese abstract page, "Limitations"); this is
  * the speculative-verify shape with per-sequence draft lengths.
  *   q_lens   int32 [batch], device, 0 <= q_lens[b] <= q_len, or NULL (all q_len).
  *            Sequence b's real query tokens are rows t < q_lens[b] of its q_len

@@ -22,7 +22,7 @@
  *
  * Ragged multi-token decode (a different number of new tokens per sequence,
  * q_lens[b] <= q_len; the pages decode one token per forward and name more
- * as a limitation, "Discussion"): token t of sequence b is a real query iff
+ * as a limitation: FlashMLA-ETAP Chinese abstract page, "Limitations"): token t of sequence b is a real query iff
  * t < q_lens[b], and then it sees j <= L_b - q_lens[b] + t when causal (its
  * q_lens[b] new tokens are the last q_lens[b] cache rows) or j < L_b; padding
  * tokens t >= q_lens[b] see no row (O = 0, LSE = -inf).
