@@ -245,17 +245,29 @@ MLA_API int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, i
  * B=32, h=128 does not fit). No call allocates memory.
  *
  * Set-up: the first call on a device (with that device current) looks up the
- * array's device address once; make that first call before any stream capture.
- * Every call shares the one array and it keeps the last call's contents (the
- * schedule rewrites everything later reads, status word included), so calls
+ * array's device address once and keeps it for the life of the process; make
+ * that first call before any stream capture. The library must not be used on a
+ * device across a cudaDeviceReset (the array then moves and the kept address is
+ * stale). Every call shares the one array and it keeps the last call's contents
+ * (the schedule rewrites everything later reads, status word included), so calls
  * that overlap on the GPU, on different streams or host threads, race: order
- * them on one stream. The device status word of these calls is internal and
- * not readable through mla_decode_read_status.
+ * them on one stream. Read the device status word of the last call (a wait that
+ * ran out, an out-of-range block-table entry) with mla_decode_static_ws_status.
  */
 MLA_API int mla_decode_fwd_static_ws(const void *q, const void *kv, const int32_t *seqlens,
                                      const int32_t *block_table, int batch, int q_len, int num_heads,
                                      int64_t kv_rows, int max_blocks, float softmax_scale, int causal,
                                      void *o, float *lse, int num_sms, void *stream);
+
+/*
+ * The device status word of the last mla_decode_fwd_static_ws call on the current
+ * device, copied to the host on `stream` (waits for that copy only): MLA_OK, or the
+ * first device-side error the call recorded (MLA_ERR_TIMEOUT, MLA_ERR_BLOCK_TABLE,
+ * MLA_ERR_INVALID_ARG). It plays the part of mla_decode_read_status for the static
+ * array, whose address callers never see. The paper has no counterpart. Allocates
+ * nothing; the same set-up rule as mla_decode_fwd_static_ws applies.
+ */
+MLA_API int mla_decode_static_ws_status(int *status_out, void *stream);
 
 /* Human-readable name of a status code. */
 MLA_API const char *mla_status_string(int status);

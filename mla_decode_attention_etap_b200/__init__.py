@@ -28,7 +28,7 @@ STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3:
 
 EXPORTS = ("mla_decode_workspace_size", "mla_decode_plan", "mla_decode_fwd", "mla_combine",
            "mla_decode_read_status", "mla_decode_plan_host", "mla_status_string", "mla_last_cuda_error",
-           "mla_decode_fwd_static_ws", "mla_decode_fwd_ragged", "mla_stream_probe", "mla_decode_fwd_fp8", "mla_form_ablation")
+           "mla_decode_fwd_static_ws", "mla_decode_static_ws_status", "mla_decode_fwd_ragged", "mla_stream_probe", "mla_decode_fwd_fp8", "mla_form_ablation")
 STATIC_WORKSPACE_BYTES = 8388608
 
 
@@ -75,6 +75,8 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_fwd_static_ws.argtypes = [vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp,
                                                vp, i32, vp]
         L.mla_decode_fwd_static_ws.restype = i32
+        L.mla_decode_static_ws_status.argtypes = [ctypes.POINTER(ctypes.c_int), vp]
+        L.mla_decode_static_ws_status.restype = i32
         L.mla_form_ablation.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp]
         L.mla_form_ablation.restype = i32
         L.mla_stream_probe.argtypes = [vp, i64, i32, vp, vp]

@@ -239,20 +239,49 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Spinning variants for the softmax warps: a non-blocking probe in a loop
 // resumes the moment the phase completes (a suspended try_wait can wake late,
 // and the slowest of the 128 threads sets the pace of the next named barrier).
+// A phase that the peer CTA completes (CLUSTER) is probed by lane 0 alone with a
+// cluster-scope acquire, and __syncwarp then orders the other lanes after it: one
+// cluster-scope acquire per warp instead of one per thread.  Call it from all 32
+// lanes of a warp.
 template <bool CLUSTER>
 __device__ __forceinline__ bool spin_phase(uint32_t bar, uint32_t parity, volatile WaitCtl *wc,
                                            int32_t *status) {
-    auto probe = [&]() { return CLUSTER ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity); };
-    if (probe()) return true;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t spin = 1;; ++spin) {
-        if (probe()) return true;
-        if ((spin & 255u) == 0) {
-            if (wc->abort) return false;
-            if (global_timer_ns() - t0 > wc->limit_ns) {
-                wc->abort = 1;
-                atomicCAS(status, 0, kStatusTimeout);
-                return false;
+    if constexpr (CLUSTER) {
+        bool ok = true;
+        if ((threadIdx.x & 31) == 0) {
+            if (!mbar_test_wait_cluster(bar, parity)) {
+                const uint64_t t0 = global_timer_ns();
+                for (uint32_t spin = 1;; ++spin) {
+                    if (mbar_test_wait_cluster(bar, parity)) break;
+                    if ((spin & 255u) == 0) {
+                        if (wc->abort) {
+                            ok = false;
+                            break;
+                        }
+                        if (global_timer_ns() - t0 > wc->limit_ns) {
+                            wc->abort = 1;
+                            atomicCAS(status, 0, kStatusTimeout);
+                            ok = false;
+                            break;
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    } else {
+        if (mbar_test_wait(bar, parity)) return true;
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t spin = 1;; ++spin) {
+            if (mbar_test_wait(bar, parity)) return true;
+            if ((spin & 255u) == 0) {
+                if (wc->abort) return false;
+                if (global_timer_ns() - t0 > wc->limit_ns) {
+                    wc->abort = 1;
+                    atomicCAS(status, 0, kStatusTimeout);
+                    return false;
+                }
             }
         }
     }

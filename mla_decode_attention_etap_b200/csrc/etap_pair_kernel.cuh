@@ -854,7 +854,14 @@ __global__ void __launch_bounds__(320, 1)
                         if (lane == 0) mbar_arrive_remote(xfree_remote);
                         // Send now only if S^T of tile k+1 is already there: with few V slots its
                         // scores can depend on step 3 of tile k, i.e. on this tile's softmax.
-                        if (k + 1 < k_total && mbar_test_wait(bar(BR::SFULL + ((k + 1) & 1)), ((k + 1) >> 1) & 1)) {
+                        // (one probe per warp, so that the warp-collective TMEM loads and the
+                        // lane-0 wait inside send_tile see the same decision in every lane)
+                        const bool next_ready =
+                            k + 1 < k_total &&
+                            __shfl_sync(0xffffffffu,
+                                        mbar_test_wait(bar(BR::SFULL + ((k + 1) & 1)), ((k + 1) >> 1) & 1) ? 1 : 0,
+                                        0) != 0;
+                        if (next_ready) {
                             send_tile(k + 1);
                             sent_next = true;
                         }

@@ -477,6 +477,24 @@ int check_static_ws_args(const void *q, const void *kv, const int32_t *seqlens, 
     return MLA_OK;
 }
 
+// Device address of g_static_ws on the current device, looked up once per device with that
+// device current (in host code the name g_static_ws is a host-side stand-in, not a device address).
+int static_ws_device_addr(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return MLA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_static_ws_mu);
+    if (!g_static_ws_addr[dev]) {
+        void *addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, g_static_ws);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+        g_static_ws_addr[dev] = addr;
+    }
+    *out = g_static_ws_addr[dev];
+    return MLA_OK;
+}
+
 }  // namespace
 
 extern "C" int mla_decode_fwd_static_ws(const void *q, const void *kv, const int32_t *seqlens,
@@ -486,26 +504,21 @@ extern "C" int mla_decode_fwd_static_ws(const void *q, const void *kv, const int
     int st = check_static_ws_args(q, kv, seqlens, block_table, batch, q_len, num_heads, kv_rows, max_blocks,
                                   softmax_scale, causal, o, lse, num_sms);
     if (st != MLA_OK) return st;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    if (dev < 0 || dev >= 64) return MLA_ERR_UNSUPPORTED;
     void *ws = nullptr;
-    {
-        std::lock_guard<std::mutex> lock(g_static_ws_mu);
-        if (!g_static_ws_addr[dev]) {
-            // In host code g_static_ws names a host-side shadow; the kernels need the device address.
-            void *addr = nullptr;
-            e = cudaGetSymbolAddress(&addr, g_static_ws);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
-            g_static_ws_addr[dev] = addr;
-        }
-        ws = g_static_ws_addr[dev];
-    }
+    st = static_ws_device_addr(&ws);
+    if (st != MLA_OK) return st;
     // The schedule rewrites the header (status word included) and the tables the
     // decode kernel reads; partial slots are written before the combine reads them.
     st = mla_decode_plan(seqlens, batch, q_len, num_heads, num_sms, ws, MLA_STATIC_WORKSPACE_BYTES, stream);
     if (st != MLA_OK) return st;
     return mla_decode_fwd(q, kv, seqlens, block_table, batch, q_len, num_heads, kv_rows, max_blocks, softmax_scale,
                           causal, o, lse, ws, MLA_STATIC_WORKSPACE_BYTES, num_sms, 0, stream);
+}
+
+extern "C" int mla_decode_static_ws_status(int *status_out, void *stream) {
+    if (!status_out) return MLA_ERR_INVALID_ARG;
+    void *ws = nullptr;
+    int st = static_ws_device_addr(&ws);
+    if (st != MLA_OK) return st;
+    return mla_decode_read_status(ws, status_out, stream);
 }

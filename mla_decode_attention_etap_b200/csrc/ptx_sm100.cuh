@@ -59,13 +59,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Non-blocking probe of a phase that the peer CTA completes (remote arrive or st.async
-// complete_tx).  The default acquire semantics are used, as for any phase completed by
-// asynchronous writes into this CTA's shared memory; a cluster-scope acquire is much slower.
+// complete_tx, both releases at cluster scope): acquire at cluster scope, so that the peer's
+// writes before its release (the st.async data, or its reads of slots it now frees) are
+// ordered before what this thread does next.
 __device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.b32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -78,7 +79,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.b32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -106,12 +107,12 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t a, ui
         ::"r"(remote_addr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(remote_bar)
         : "memory");
 }
-// Arrive on a barrier of another CTA of the cluster that only says "your slots here may be
-// overwritten": the reads of those slots precede it in program order, and the default
-// (release, CTA scope) semantics suffice, as for a consumer releasing a stage that a peer
-// refills asynchronously.  A cluster-scope release costs about a microsecond here.
+// Arrive on a barrier of another CTA of the cluster ("your slots here may be overwritten" or
+// "this data is ready"): a release at cluster scope, which orders this thread's earlier reads
+// and writes (and, after a __syncwarp or a barrier, its warp's or CTA's) before the peer's
+// cluster-scope acquire of that phase.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
-    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");

@@ -236,3 +236,18 @@ def test_cuda_graph_replay_matches_eager():
         torch.cuda.synchronize()
         assert torch.equal(o, o_eager) and torch.equal(lse, l_eager)
     assert dec.status() == 0
+
+
+def test_precision_margin_over_seeds_and_lengths():
+    """The FP8 path's error sits close to the bar (bf16 rounding of O alone takes ~1.65e-3 of the
+    2e-3): sweep 8 seeds x lengths {333, 1024, 4096} (one sequence each, 16 heads) and require the
+    worst RMSE / RMS(O_ref) to stay at or below 1.9e-3, a 5 % margin under the parity bar."""
+    worst = 0.0
+    for seed in range(8):
+        for L in (333, 1024, 4096):
+            w = fp8(1, 16, [L], seed=900 + 10 * seed + L % 7)
+            o, lse, st, _ = run_cuda(w)
+            assert st == 0
+            m = assert_parity(o, lse, *run_oracle(w), what=f"fp8 seed={seed} L={L}")
+            worst = max(worst, m["rmse_rel"])
+    assert worst <= 1.9e-3, worst

@@ -402,3 +402,31 @@ def test_form_ablation_runs(heads):
             assert int(err.item()) == 0
             # at least 8 tiles x 16 MMAs at >= 8 cycles each
             assert int(cycles.min().item()) > 8 * 16 * 8
+
+
+@pytest.mark.parametrize("heads,q_len,causal,lens", [(16, 1, False, [6000, 3000, 9000, 500]),
+                                                     (16, 4, True, [3000, 2000, 700, 4100]),
+                                                     (128, 1, False, [2500, 900])])
+def test_repeated_decodes_are_bitwise_identical(heads, q_len, causal, lens):
+    """Stress of the cross-CTA hand-offs (score exchange, slot release, pair merge): 200 plan +
+    decode calls on one input must all give the bits of the first; a torn exchange would show up
+    as a one-off difference.  The first result is also checked against the oracle."""
+    from mla_decode_attention_etap_b200 import MlaDecoder
+    w = W.make_workload(len(lens), heads, lens, q_len=q_len, causal=causal, seed=90 + heads + q_len)
+    dev = torch.device("cuda")
+    q, kv, sl = w.q.to(dev), w.kv.to(dev), w.seqlens.to(dev)
+    dec = MlaDecoder(w.batch, w.q_len, w.num_heads, device=dev)
+    o0 = lse0 = None
+    bad = 0
+    for i in range(200):
+        dec.plan(sl)
+        o, lse = dec.fwd(q, kv, sl, None, w.softmax_scale, w.causal)
+        if o0 is None:
+            o0, lse0 = o.clone(), lse.clone()
+        elif not (torch.equal(o.view(torch.int16), o0.view(torch.int16)) and
+                  torch.equal(lse.view(torch.int32), lse0.view(torch.int32))):
+            bad += 1
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    assert bad == 0, f"{bad} of 199 repeats differ from the first"
+    assert_parity(o0.float().cpu().numpy(), lse0.cpu().numpy(), *run_oracle(w), what="repeat stress")
