@@ -239,10 +239,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Spinning variants for the softmax warps: a non-blocking probe in a loop
 // resumes the moment the phase completes (a suspended try_wait can wake late,
 // and the slowest of the 128 threads sets the pace of the next named barrier).
-// A phase that the peer CTA completes (CLUSTER) is probed by lane 0 alone with a
-// cluster-scope acquire, and __syncwarp then orders the other lanes after it: one
-// cluster-scope acquire per warp instead of one per thread.  Call it from all 32
-// lanes of a warp.
+// A phase that the peer CTA completes (CLUSTER) is polled by lane 0 alone with relaxed
+// cluster-scope probes; a restricted acquire fence then synchronises with the peer's release,
+// and __syncwarp orders the other lanes after lane 0.  Call it from all 32 lanes of a warp.
 template <bool CLUSTER>
 __device__ __forceinline__ bool spin_phase(uint32_t bar, uint32_t parity, volatile WaitCtl *wc,
                                            int32_t *status) {
@@ -267,6 +266,7 @@ __device__ __forceinline__ bool spin_phase(uint32_t bar, uint32_t parity, volati
                     }
                 }
             }
+            fence_acquire_cluster_smem();
         }
         __syncwarp();
         return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -282,24 +282,6 @@ __device__ __forceinline__ bool spin_phase(uint32_t bar, uint32_t parity, volati
                     atomicCAS(status, 0, kStatusTimeout);
                     return false;
                 }
-            }
-        }
-    }
-}
-
-// Bounded wait on a phase completed by the peer CTA of the cluster.
-__device__ __forceinline__ bool wait_phase_cluster(uint32_t bar, uint32_t parity, volatile WaitCtl *wc,
-                                                   int32_t *status) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    for (uint32_t spin = 1;; ++spin) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if ((spin & 63u) == 0) {
-            if (wc->abort) return false;
-            if (global_timer_ns() - t0 > wc->limit_ns) {
-                wc->abort = 1;
-                atomicCAS(status, 0, kStatusTimeout);
-                return false;
             }
         }
     }
