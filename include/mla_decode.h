@@ -62,7 +62,7 @@ enum {
     MLA_PAGE_SIZE = 64,  /* tokens per page of a paged cache */
     MLA_MAX_BATCH = 65536,
     MLA_MAX_COLUMNS = 1024, /* max q_len * num_heads */
-    MLA_STATIC_WORKSPACE_BYTES = 8388608 /* scratch of mla_decode_fwd_static_ws: 8 MiB per GPU */
+    MLA_STATIC_WORKSPACE_BYTES = 16777216 /* scratch of mla_decode_fwd_static_ws: 16 MiB per GPU */
 };
 
 /* Flags for mla_decode_fwd. */
@@ -194,6 +194,28 @@ MLA_API int mla_combine(const void *workspace, int batch, int q_len, int num_hea
 MLA_API int mla_stream_probe(const void *kv, int64_t rows, int units, int32_t *err, void *stream);
 
 /*
+ * Measurement helper, not part of the decode (the pages have no counterpart): mla_decode_fwd
+ * (flags 0) that also records when each role of the two CTAs of cluster 0 reached its events, so
+ * that the pipeline of the M = 256 kernel (bf16 cache, q_len*h > 16) can be read off one launch.
+ *   trace      device uint64 [2 CTAs][5 roles][trace_cap], then [num_sms][4]: 8-byte aligned,
+ *              zeroed by the caller; roles: 0 K-tile producer, 1 step-1 MMA issuer (CTA 0 only),
+ *              2 value producer, 3 softmax, 4 step-3 MMA issuer (CTA 0 only).  The trailing
+ *              rows hold each CTA's %globaltimer (ns) at entry, start of work (the plan read),
+ *              end of work and exit.
+ *              Entry = (event code << 56) | (index << 40) | (%globaltimer ns mod 2^40); a role
+ *              stops recording after trace_cap events.  The event codes are listed in
+ *              etap_duo_kernel.cuh.  Other shapes run the untraced kernels and leave it as it is.
+ *   trace_cap  1 .. 2^20
+ * All other arguments, results and errors as for mla_decode_fwd.  The stamps cost a few
+ * instructions per event in those four threads.
+ */
+MLA_API int mla_decode_fwd_trace(const void *q, const void *kv, const int32_t *seqlens, const int32_t *block_table,
+                                 int batch, int q_len, int num_heads, int64_t kv_rows, int max_blocks,
+                                 float softmax_scale, int causal, void *o, float *lse, void *workspace,
+                                 size_t workspace_bytes, int num_sms, unsigned long long *trace, int trace_cap,
+                                 void *stream);
+
+/*
  * Measurement helper for the pages' argument for the transposed form (FlashMLA-ETAP technical
  * summary, "Problem Statement": with few heads the untransposed S = Q K^T pads the query heads up
  * to the tensor core's minimum M; "Methodology": S^T = K Q^T puts the KV rows on M instead).  Issues,
@@ -217,15 +239,21 @@ MLA_API int mla_form_ablation(int form, int heads, int streams, int tiles, int c
 MLA_API int mla_decode_read_status(const void *workspace, int *status_out, void *stream);
 
 /*
- * Host mirror of the split-KV schedule, for testing and for callers that
- * want to inspect it. seqlens is a HOST int32[batch]. Writes, when the
- * pointers are non-NULL:
- *   cta_ranges  int32[num_ctas*2]  flattened tile range [begin, end) of each CTA
- *   seq_info    int32[batch*4]     per sequence: tile count, first CTA, number of splits, partial slot offset
- * and returns the number of CTAs per column group (num_ctas) through *num_ctas_out.
+ * Host mirror of the split-KV schedules, for testing and for callers that want to inspect
+ * them. seqlens is a HOST int32[batch]. `schedule` 0 is the one mla_decode_fwd_fp8 uses (and
+ * mla_decode_fwd for q_len*h <= 16): 128-row units, column groups of 16 or 32. `schedule` 1
+ * is the one mla_decode_fwd uses: for q_len*h > 16, 256-row units (one 128-row tile per CTA of
+ * a pair) and column groups of 64, or of 128 when q_len*h > 64 and every nonempty sequence
+ * holds at least 8192 rows (the plan picks this on the device from the same lengths); for
+ * q_len*h <= 16 it is schedule 0. Writes, when the pointers are non-NULL:
+ *   cta_ranges  int32[num_ctas*2]  flattened unit range [begin, end) of each work unit
+ *   seq_info    int32[batch*4]     per sequence: unit count, first work unit, number of splits, partial slot offset
+ * and returns the work units per column group, the column groups, the rows per unit and the
+ * columns per group through the output pointers (each may be NULL).
  */
 MLA_API int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, int num_heads, int num_sms,
-                         int32_t *cta_ranges, int32_t *seq_info, int *num_ctas_out, int *num_groups_out);
+                                 int schedule, int32_t *cta_ranges, int32_t *seq_info, int *num_ctas_out,
+                                 int *num_groups_out, int *unit_rows_out, int *group_cols_out);
 
 /*
  * The whole decode (schedule, ETAP decode, combine) for callers that cannot
@@ -241,8 +269,8 @@ MLA_API int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, i
  * Arguments are those of mla_decode_fwd minus the workspace and flags.
  * Returns MLA_ERR_WORKSPACE, launching nothing, when
  * mla_decode_workspace_size(batch, q_len, num_heads, num_sms) exceeds
- * MLA_STATIC_WORKSPACE_BYTES (e.g. B=16, h=16 needs about 5.4 MB on 148 SMs;
- * B=32, h=128 does not fit). No call allocates memory.
+ * MLA_STATIC_WORKSPACE_BYTES (on 148 SMs: B=16, h=16 needs about 3 MB and
+ * B=16, q_len=4, h=16 about 12 MB; B=32, h=128 does not fit). No call allocates memory.
  *
  * Set-up: the first call on a device (with that device current) looks up the
  * array's device address once and keeps it for the life of the process; make

@@ -28,8 +28,9 @@ STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3:
 
 EXPORTS = ("mla_decode_workspace_size", "mla_decode_plan", "mla_decode_fwd", "mla_combine",
            "mla_decode_read_status", "mla_decode_plan_host", "mla_status_string", "mla_last_cuda_error",
-           "mla_decode_fwd_static_ws", "mla_decode_static_ws_status", "mla_decode_fwd_ragged", "mla_stream_probe", "mla_decode_fwd_fp8", "mla_form_ablation")
-STATIC_WORKSPACE_BYTES = 8388608
+           "mla_decode_fwd_static_ws", "mla_decode_static_ws_status", "mla_decode_fwd_ragged", "mla_stream_probe", "mla_decode_fwd_fp8", "mla_form_ablation",
+           "mla_decode_fwd_trace")
+STATIC_WORKSPACE_BYTES = 16777216
 
 
 class MlaError(RuntimeError):
@@ -67,8 +68,8 @@ def lib() -> ctypes.CDLL:
         L.mla_combine.restype = i32
         L.mla_decode_read_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
         L.mla_decode_read_status.restype = i32
-        L.mla_decode_plan_host.argtypes = [vp, i32, i32, i32, i32, vp, vp, ctypes.POINTER(ctypes.c_int),
-                                           ctypes.POINTER(ctypes.c_int)]
+        ip = ctypes.POINTER(ctypes.c_int)
+        L.mla_decode_plan_host.argtypes = [vp, i32, i32, i32, i32, i32, vp, vp, ip, ip, ip, ip]
         L.mla_decode_plan_host.restype = i32
         L.mla_status_string.argtypes = [i32]
         L.mla_status_string.restype = ctypes.c_char_p
@@ -79,6 +80,9 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_static_ws_status.restype = i32
         L.mla_form_ablation.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp]
         L.mla_form_ablation.restype = i32
+        L.mla_decode_fwd_trace.argtypes = [vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp, vp, vp,
+                                           sz, i32, vp, i32, vp]
+        L.mla_decode_fwd_trace.restype = i32
         L.mla_stream_probe.argtypes = [vp, i64, i32, vp, vp]
         L.mla_stream_probe.restype = i32
         L.mla_last_cuda_error.argtypes = []
@@ -215,6 +219,70 @@ def mla_decode_fwd_fp8(q, kv8, kv_scale, seqlens, block_table, softmax_scale, ca
            "mla_decode_fwd_fp8")
 
 
+TRACE_ROLES = ("K-tile producer", "step-1 issuer", "value producer", "softmax", "step-3 issuer")
+
+
+def mla_decode_fwd_trace(q, kv, seqlens, block_table, softmax_scale, causal, o, lse, workspace, n_sms, trace,
+                         stream=None) -> None:
+    """mla_decode_fwd that also records the event stamps of cluster 0's roles into ``trace`` (int64 device
+    tensor of 2 * 5 * cap + 8 * n_sms elements, zeroed by the caller, made by trace_buffer()); see
+    decode_trace_events() and decode_trace_spans()."""
+    _require_cuda(q, "q")
+    check_decode_args(q, kv, seqlens, block_table, o, lse, workspace)
+    _require(trace, "trace", torch.int64, q.device, dim=1)
+    cap = (trace.numel() - 8 * n_sms) // (2 * len(TRACE_ROLES))
+    if cap < 1 or trace.numel() != 2 * len(TRACE_ROLES) * cap + 8 * n_sms:
+        raise ValueError("trace: use trace_buffer(cap, n_sms)")
+    B, q_len, h, _ = q.shape
+    if block_table is not None:
+        kv_rows, max_blocks = kv.shape[0] * kv.shape[1], block_table.shape[1]
+    else:
+        kv_rows, max_blocks = kv.shape[1], 0
+    _check(lib().mla_decode_fwd_trace(_ptr(q), _ptr(kv), _ptr(seqlens), _ptr(block_table), B, q_len, h, kv_rows,
+                                      max_blocks, float(softmax_scale), int(bool(causal)), _ptr(o), _ptr(lse),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(), n_sms,
+                                      _ptr(trace), cap, _stream(stream)), "mla_decode_fwd_trace")
+
+
+def trace_buffer(cap: int, n_sms: int, device=None):
+    """A zeroed trace buffer for mla_decode_fwd_trace: [2 CTAs][5 roles][cap] stamps, then [n_sms][4]."""
+    return torch.zeros(2 * len(TRACE_ROLES) * cap + 8 * n_sms, dtype=torch.int64, device=device)
+
+
+def decode_trace_spans(trace, n_sms: int):
+    """Trace buffer -> [n_sms, 4] (entry, start of work, end of work, exit) ns of every CTA, relative to the
+    earliest entry (rows of CTAs that did not run stay 0)."""
+    import numpy as np
+    t = np.asarray(trace.cpu() if isinstance(trace, torch.Tensor) else trace).astype(np.int64)
+    sp = t[len(t) - 8 * n_sms:].reshape(n_sms, 8).copy()
+    live = sp[:, 0] > 0
+    if live.any():
+        sp[live] -= sp[live, 0].min()
+    return sp
+
+
+def decode_trace_events(trace, n_sms: int = None):
+    """Trace buffer -> list of (cta, role, code, index, t_ns) sorted by time (t relative to the first stamp)."""
+    import numpy as np
+    t = np.asarray(trace.cpu() if isinstance(trace, torch.Tensor) else trace).astype(np.uint64)
+    if n_sms is not None:
+        t = t[:len(t) - 8 * n_sms]
+    t = t.reshape(2, len(TRACE_ROLES), -1)
+    out = []
+    for cta in range(t.shape[0]):
+        for role in range(t.shape[1]):
+            for w in t[cta, role]:
+                w = int(w)
+                if w == 0:
+                    break
+                out.append((cta, role, w >> 56, (w >> 40) & 0xFFFF, w & 0xFFFFFFFFFF))
+    if not out:
+        return out
+    t0 = min(e[4] for e in out)
+    out = [(c, r, k, i, ts - t0) for c, r, k, i, ts in out]
+    return sorted(out, key=lambda e: e[4])
+
+
 def mla_stream_probe(kv, units: int, err, stream=None) -> None:
     """Stream ``kv`` ([..., 576] bf16, rows a multiple of 128) with the decode's TMA read pattern and
     no computation (a bandwidth probe).  ``err``: int32 device tensor [1], zeroed by the caller."""
@@ -252,19 +320,22 @@ def mla_decode_read_status(workspace, stream=None) -> int:
     return int(out.value)
 
 
-def mla_decode_plan_host(seqlens, q_len: int, num_heads: int, n_sms: int):
-    """Host mirror of the schedule -> (cta_ranges [ctas, 2], seq_info [B, 4], num_ctas, num_groups)."""
+def mla_decode_plan_host(seqlens, q_len: int, num_heads: int, n_sms: int, schedule: int = 1):
+    """Host mirror of a schedule -> (cta_ranges [ctas, 2], seq_info [B, 4], num_ctas, num_groups, unit_rows,
+    group_cols).  schedule 1: the one mla_decode_fwd (bf16 cache) uses; 0: the one mla_decode_fwd_fp8 uses."""
     import numpy as np
     sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
-    nct, ngr = ctypes.c_int(0), ctypes.c_int(0)
-    _check(lib().mla_decode_plan_host(sl.ctypes.data_as(ctypes.c_void_p), sl.size, q_len, num_heads, n_sms, None,
-                                      None, ctypes.byref(nct), ctypes.byref(ngr)), "mla_decode_plan_host")
+    nct, ngr, urows, gcols = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().mla_decode_plan_host(sl.ctypes.data_as(ctypes.c_void_p), sl.size, q_len, num_heads, n_sms, schedule,
+                                      None, None, ctypes.byref(nct), ctypes.byref(ngr), ctypes.byref(urows),
+                                      ctypes.byref(gcols)), "mla_decode_plan_host")
     ranges = np.zeros((nct.value, 2), np.int32)
     info = np.zeros((sl.size, 4), np.int32)
-    _check(lib().mla_decode_plan_host(sl.ctypes.data_as(ctypes.c_void_p), sl.size, q_len, num_heads, n_sms,
+    _check(lib().mla_decode_plan_host(sl.ctypes.data_as(ctypes.c_void_p), sl.size, q_len, num_heads, n_sms, schedule,
                                       ranges.ctypes.data_as(ctypes.c_void_p), info.ctypes.data_as(ctypes.c_void_p),
-                                      ctypes.byref(nct), ctypes.byref(ngr)), "mla_decode_plan_host")
-    return ranges, info, nct.value, ngr.value
+                                      ctypes.byref(nct), ctypes.byref(ngr), ctypes.byref(urows), ctypes.byref(gcols)),
+           "mla_decode_plan_host")
+    return ranges, info, nct.value, ngr.value, urows.value, gcols.value
 
 
 class MlaDecoder:

@@ -60,6 +60,27 @@ struct DecodeParams {
     int32_t *counters;  // [batch][groups][2]: split CTAs done per (sequence, column group, rank)
     int slots;          // partial slots (stride between the two ranks' LSE partial arrays)
     int fuse_merge;     // the last split CTA of a sequence merges the partials (no combine launch)
+    unsigned long long *trace;  // measurement: event stamps of cluster 0's roles, or NULL
+    int trace_cap;              // stamps per (CTA, role) in `trace`
+};
+
+// Event stamps for the tracing entry point: (code << 56) | (index << 40) | (globaltimer ns mod 2^40),
+// written by one thread per (CTA, role) of cluster 0 into its own row of the trace buffer.
+enum : int { kTraceRoles = 5 };
+struct TraceRow {
+    unsigned long long *row;
+    int n, cap;
+    __device__ void init(const DecodeParams &p, int role) {
+        n = 0;
+        cap = p.trace_cap;
+        row = (p.trace && blockIdx.x < 2) ? p.trace + ((size_t)blockIdx.x * kTraceRoles + role) * (size_t)cap : nullptr;
+    }
+    __device__ __forceinline__ void put(int code, int index) {
+        if (row && n < cap) {
+            row[n++] = ((unsigned long long)code << 56) | ((unsigned long long)(index & 0xFFFF) << 40) |
+                       (global_timer_ns() & 0xFFFFFFFFFFull);
+        }
+    }
 };
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA abort
@@ -71,6 +92,24 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
     for (uint32_t spin = 1;; ++spin) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((spin & 63u) == 0) {
+            if (wc->abort) return false;
+            if (global_timer_ns() - t0 > wc->limit_ns) {
+                wc->abort = 1;
+                atomicCAS(status, 0, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+// Bounded wait that polls instead of suspending: for phases that the other CTA of a pair completes
+// (a multicast tcgen05.commit, a remote arrive), where a suspended try_wait can resume microseconds
+// late.  Same abort and timeout handling as wait_phase.
+__device__ __forceinline__ bool poll_phase(uint32_t bar, uint32_t parity, volatile WaitCtl *wc, int32_t *status) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((spin & 255u) == 0) {
             if (wc->abort) return false;
             if (global_timer_ns() - t0 > wc->limit_ns) {
                 wc->abort = 1;

@@ -309,7 +309,9 @@ __global__ void __launch_bounds__(320, 1)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // The schedule must come from a plan for this same grid (uniform in the whole cluster).
-    const bool plan_ok = p.ws[kHdrCtas] == p.ctas && p.ws[kHdrGroups] == p.groups && p.ws[kHdrBatch] == p.batch;
+    const bool plan_ok = p.ws[kHdrPair + kSchCtas] == p.ctas && p.ws[kHdrPair + kSchGroups] == p.groups &&
+                         p.ws[kHdrBatch] == p.batch;
+    if (blockIdx.x == 0 && threadIdx.x == 0) p.ws[kHdrSchedUsed] = 0;  // the partials follow the pair schedule
 
     const int32_t *ranges = p.ws + p.cta_ranges_off;
     const int32_t *tile_off = p.ws + p.tile_off_off;

@@ -14,6 +14,7 @@
 
 #include "mla_decode.h"
 #include "etap_pair_kernel.cuh"
+#include "etap_duo_kernel.cuh"
 #include "plan_combine_kernels.cuh"
 #include "plan_core.h"
 #include "form_ablation.cuh"
@@ -105,6 +106,9 @@ int ensure_smem_attr() {
         e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg32E4>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::PairCfg32E4::SMEM_ALLOC);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        e = cudaFuncSetAttribute(mla::etap_duo_kernel<mla::DuoCfg64, mla::DuoCfg128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::kDuoSmemAlloc);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         done[dev] = true;
     }
     return MLA_OK;
@@ -133,6 +137,26 @@ cudaError_t launch_pair(const CUtensorMap &tm_q, const CUtensorMap &tm_kv, const
     return cudaLaunchKernelEx(&cfg, mla::etap_pair_kernel<C>, tm_q, tm_kv, tm_qr, tm_kvr, p);
 }
 
+// The duo kernel: one 2-CTA cluster per (work unit, column group); the grid covers the largest
+// grouping the plan may pick (the clusters past the plan's own count find no work).
+cudaError_t launch_duo(const mla::DuoMaps &maps, const mla::DecodeParams &p, int clusters, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters, 1, 1);
+    cfg.blockDim = dim3(mla::kDuoThreads, 1, 1);
+    cfg.dynamicSmemBytes = mla::kDuoSmemAlloc;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, mla::etap_duo_kernel<mla::DuoCfg64, mla::DuoCfg128>, maps, p);
+}
+
 }  // namespace
 
 extern "C" {
@@ -158,18 +182,33 @@ size_t mla_decode_workspace_size(int batch, int q_len, int num_heads, int num_sm
     return mla::ws_layout(batch, q_len, num_heads, num_sms).total;
 }
 
-int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, int num_heads, int num_sms,
-                         int32_t *cta_ranges, int32_t *seq_info, int *num_ctas_out, int *num_groups_out) {
+int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, int num_heads, int num_sms, int schedule,
+                         int32_t *cta_ranges, int32_t *seq_info, int *num_ctas_out, int *num_groups_out,
+                         int *unit_rows_out, int *group_cols_out) {
     int st = check_shape(batch, q_len, num_heads, num_sms);
     if (st != MLA_OK) return st;
-    if (!seqlens) return MLA_ERR_INVALID_ARG;
+    if (!seqlens || (schedule != 0 && schedule != 1)) return MLA_ERR_INVALID_ARG;
     const mla::WsLayout lay = mla::ws_layout(batch, q_len, num_heads, num_sms);
+    const int ncols = q_len * num_heads;
+    // schedule 1 (the bf16 cache) is the duo schedule when the shape has one, else the pair schedule
+    const bool duo = schedule == 1 && lay.has_duo;
+    int ctas = lay.ctas, groups = lay.groups, unit_rows = mla::kTileRows, gcols = mla::group_cols(ncols);
+    if (duo) {
+        int mn = 0;
+        for (int b = 0; b < batch; ++b)
+            if (seqlens[b] > 0 && (mn == 0 || seqlens[b] < mn)) mn = seqlens[b];
+        const int mode = mla::duo_mode(ncols, mn);
+        groups = mla::duo_groups(ncols, mode);
+        ctas = mla::num_ctas(num_sms, groups);
+        unit_rows = mla::kDuoRows;
+        gcols = mla::duo_group_cols(mode);
+    }
     int64_t total = 0;
-    for (int b = 0; b < batch; ++b) total += mla::tiles_of(seqlens[b]);
+    for (int b = 0; b < batch; ++b) total += mla::units_of(seqlens[b], unit_rows);
     if (total > INT32_MAX) return MLA_ERR_UNSUPPORTED;
-    const int used = mla::used_ctas(total, lay.ctas);
+    const int used = mla::used_ctas(total, ctas);
     if (cta_ranges)
-        for (int c = 0; c < lay.ctas; ++c) {
+        for (int c = 0; c < ctas; ++c) {
             cta_ranges[2 * c] = (int32_t)mla::cta_begin(total, used, c);
             cta_ranges[2 * c + 1] = (int32_t)mla::cta_begin(total, used, c + 1);
         }
@@ -177,7 +216,7 @@ int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, int num_h
         int64_t off = 0;
         int slots = 0;
         for (int b = 0; b < batch; ++b) {
-            const int64_t t0 = off, t1 = off + mla::tiles_of(seqlens[b]);
+            const int64_t t0 = off, t1 = off + mla::units_of(seqlens[b], unit_rows);
             int first = -1, nsplit = 0;
             if (t1 > t0) {
                 first = mla::cta_of(total, used, t0);
@@ -191,8 +230,10 @@ int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, int num_h
             off = t1;
         }
     }
-    if (num_ctas_out) *num_ctas_out = lay.ctas;
-    if (num_groups_out) *num_groups_out = lay.groups;
+    if (num_ctas_out) *num_ctas_out = ctas;
+    if (num_groups_out) *num_groups_out = groups;
+    if (unit_rows_out) *unit_rows_out = unit_rows;
+    if (group_cols_out) *group_cols_out = gcols;
     return MLA_OK;
 }
 
@@ -216,7 +257,7 @@ int mla_decode_plan(const int32_t *seqlens, int batch, int q_len, int num_heads,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, mla::plan_kernel, seqlens, batch, lay.ctas, lay.groups, q_len * num_heads,
+    cudaError_t e = cudaLaunchKernelEx(&cfg, mla::plan_kernel, seqlens, batch, q_len * num_heads, num_sms,
                                        reinterpret_cast<int32_t *>(workspace), lay);
     if (e != cudaSuccess) return cuda_fail(e, "plan_kernel launch");
     e = cudaGetLastError();
@@ -259,7 +300,8 @@ namespace {
 int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const int32_t *seqlens,
                     const int32_t *q_lens, const int32_t *block_table, int batch, int q_len, int num_heads,
                     int64_t kv_rows, int max_blocks, float softmax_scale, int causal, void *o, float *lse,
-                    void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream) {
+                    void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream,
+                    unsigned long long *trace = nullptr, int trace_cap = 0) {
     const bool fp8 = kv_scale != nullptr;
     int st = check_shape(batch, q_len, num_heads, num_sms);
     if (st != MLA_OK) return st;
@@ -288,6 +330,8 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
     CUtensorMap tm_q, tm_kv, tm_qr, tm_kvr;
     const int ng = mla::group_cols(ncols);
     const uint64_t kv_total_rows = paged ? (uint64_t)kv_rows : (uint64_t)batch * kv_rows;
+    // the bf16 cache with more than 16 query columns runs the M = 256 kernel on the duo schedule
+    const bool duo = !fp8 && lay.has_duo;
     if (fp8) {
         // the E4M3 kernel quantises Q itself (no Q maps): 128-code boxes of the latent part, 64-code rope boxes
         st = encode_rows_576(&tm_kv, kv, kv_total_rows, 64, 128, 1);
@@ -296,6 +340,8 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
         if (st != MLA_OK) return st;
         tm_q = tm_kv;
         tm_qr = tm_kvr;
+    } else if (duo) {
+        tm_q = tm_qr = tm_kvr = CUtensorMap{};
     } else {
         st = encode_rows_576(&tm_q, q, (uint64_t)batch * ncols, (uint32_t)ng);
         if (st != MLA_OK) return st;
@@ -332,12 +378,14 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.wait_limit_ns = (flags & MLA_FLAG_TEST_EXPIRE_WAITS) ? mla::kTestWaitLimitNs : mla::kWaitLimitNs;
     p.withhold_q = (flags & MLA_FLAG_TEST_EXPIRE_WAITS) ? 1 : 0;
-    p.cta_ranges_off = (int)(lay.cta_ranges / 4);
-    p.tile_off_off = (int)(lay.tile_off / 4);
-    p.seq_info_off = (int)(lay.seq_info / 4);
-    p.cta_seq_off = (int)(lay.cta_seq / 4);
-    p.counters = reinterpret_cast<int32_t *>(ws + lay.counters);
+    p.cta_ranges_off = (int)(lay.pair.cta_ranges / 4);
+    p.tile_off_off = (int)(lay.pair.tile_off / 4);
+    p.seq_info_off = (int)(lay.pair.seq_info / 4);
+    p.cta_seq_off = (int)(lay.pair.cta_seq / 4);
+    p.counters = reinterpret_cast<int32_t *>(ws + lay.pair.counters);
     p.slots = lay.slots;
+    p.trace = trace;
+    p.trace_cap = trace ? trace_cap : 0;
     // splits of a sequence are at most the work units (CTA pairs per column group)
     const int max_splits = fp8 ? (ng == 16 ? mla::PairCfg16E4::MERGE_MAX_SPLITS : mla::PairCfg32E4::MERGE_MAX_SPLITS)
                                : (ng == 16 ? mla::PairCfg16::MERGE_MAX_SPLITS : mla::PairCfg32::MERGE_MAX_SPLITS);
@@ -345,8 +393,37 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
     p.fuse_merge = ((flags & MLA_FLAG_SKIP_COMBINE) || separate_combine) ? 0 : 1;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int clusters = lay.ctas * lay.groups;
     cudaError_t e;
+    if (duo) {
+        mla::DuoMaps maps;
+        st = encode_rows_576(&maps.q32, q, (uint64_t)batch * ncols, 32);
+        if (st != MLA_OK) return st;
+        st = encode_rows_576(&maps.q64, q, (uint64_t)batch * ncols, 64);
+        if (st != MLA_OK) return st;
+        st = encode_rows_576(&maps.kv, kv, kv_total_rows, 64);
+        if (st != MLA_OK) return st;
+        // the plan picks the grouping on the device (see plan_core.h); the kernel reads it from the header
+        p.ctas = lay.duo.ctas_max;
+        p.groups = lay.duo.groups_max;
+        p.cta_ranges_off = (int)(lay.duo.cta_ranges / 4);
+        p.tile_off_off = (int)(lay.duo.tile_off / 4);
+        p.seq_info_off = (int)(lay.duo.seq_info / 4);
+        p.cta_seq_off = (int)(lay.duo.cta_seq / 4);
+        p.counters = reinterpret_cast<int32_t *>(ws + lay.duo.counters);
+        p.fuse_merge = (flags & MLA_FLAG_SKIP_COMBINE) ? 0 : 1;
+        int clusters = 0;
+        for (int mode = 0; mode < 2; ++mode) {
+            if (mode == 1 && !mla::duo_mode1_possible(ncols)) break;
+            const int g = mla::duo_groups(ncols, mode), c = mla::num_ctas(num_sms, g) * g;
+            if (c > clusters) clusters = c;
+        }
+        e = launch_duo(maps, p, clusters, s);
+        if (e != cudaSuccess) return cuda_fail(e, "etap_duo_kernel launch");
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "etap_duo_kernel launch");
+        return MLA_OK;
+    }
+    const int clusters = lay.ctas * lay.groups;
     if (fp8)
         e = ng == 16 ? launch_pair<mla::PairCfg16E4>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s)
                      : launch_pair<mla::PairCfg32E4>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s);
@@ -380,6 +457,17 @@ int mla_decode_fwd_fp8(const void *q, const void *kv8, const float *kv_scale, co
     return decode_fwd_impl(q, kv8, kv_scale, seqlens, q_lens, block_table, batch, q_len, num_heads, kv_rows,
                            max_blocks, softmax_scale, causal, o, lse, workspace, workspace_bytes, num_sms, flags,
                            stream);
+}
+
+int mla_decode_fwd_trace(const void *q, const void *kv, const int32_t *seqlens, const int32_t *block_table, int batch,
+                         int q_len, int num_heads, int64_t kv_rows, int max_blocks, float softmax_scale, int causal,
+                         void *o, float *lse, void *workspace, size_t workspace_bytes, int num_sms,
+                         unsigned long long *trace, int trace_cap, void *stream) {
+    if (!trace || trace_cap < 1 || trace_cap > (1 << 20)) return MLA_ERR_INVALID_ARG;
+    if (!aligned(trace, 8)) return MLA_ERR_ALIGNMENT;
+    return decode_fwd_impl(q, kv, nullptr, seqlens, nullptr, block_table, batch, q_len, num_heads, kv_rows, max_blocks,
+                           softmax_scale, causal, o, lse, workspace, workspace_bytes, num_sms, 0, stream, trace,
+                           trace_cap);
 }
 
 int mla_stream_probe(const void *kv, int64_t rows, int units, int32_t *err, void *stream) {

@@ -38,37 +38,40 @@ __device__ __forceinline__ int64_t block_exclusive_scan(int64_t x, int64_t *smem
     return base + incl - x;
 }
 
-// One CTA: tile prefix sums, per-CTA flattened ranges, per-sequence split info, and
-// zeroed merge counters.  Writes the header (and clears the status word) so that the
-// decode kernel can check that it runs on a plan for its own grid.  kPlanThreads
-// threads; thread i owns the consecutive sequences [i*per, (i+1)*per).
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t *__restrict__ seqlens, int batch, int ctas,
-                                                            int groups, int ncols, int32_t *__restrict__ ws,
-                                                            WsLayout lay) {
-    // Launched as a programmatic dependent: nothing is read (seqlens may come from the
-    // preceding kernel) or written (that kernel may still read the workspace) before it
-    // completes.  Then the decode kernel may start its prologue: it waits for this grid in
-    // turn before reading the workspace.  Both are no-ops without programmatic launch.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    __shared__ int64_t scan_smem[32];
-    int32_t *tile_off = ws + lay.tile_off / 4;
-    int32_t *ranges = ws + lay.cta_ranges / 4;
-    int32_t *seq_info = ws + lay.seq_info / 4;
-    int32_t *counters = ws + lay.counters / 4;
-    int32_t *cta_seq = ws + lay.cta_seq / 4;
-    const int per = (batch + kPlanThreads - 1) / kPlanThreads;
-    const int b0 = min(batch, (int)threadIdx.x * per), b1 = min(batch, b0 + per);
-    // flattened tile offsets: exclusive prefix sum of tiles per sequence
+// Minimum of one int per thread over the block (all threads call it).
+__device__ __forceinline__ int block_min(int x, int *smem32) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+#pragma unroll
+    for (int d = 16; d >= 1; d >>= 1) x = min(x, __shfl_xor_sync(0xffffffffu, x, d));
+    if (lane == 0) smem32[warp] = x;
+    __syncthreads();
+    int r = smem32[0];
+    for (int w = 1; w < nwarps; ++w) r = min(r, smem32[w]);
+    __syncthreads();
+    return r;
+}
+
+// One schedule: unit prefix sums, per-CTA flattened ranges, per-sequence split info and
+// zeroed merge counters, plus its header words.  Every thread of the block calls it; thread i
+// owns the consecutive sequences [b0, b1).
+__device__ void plan_schedule(const int32_t *__restrict__ seqlens, int batch, int b0, int b1, int ctas, int groups,
+                              int unit_rows, int gcols, int mode, int32_t *__restrict__ ws, const Sched &sc, int hdr,
+                              int64_t *scan_smem) {
+    int32_t *tile_off = ws + sc.tile_off / 4;
+    int32_t *ranges = ws + sc.cta_ranges / 4;
+    int32_t *seq_info = ws + sc.seq_info / 4;
+    int32_t *counters = ws + sc.counters / 4;
+    int32_t *cta_seq = ws + sc.cta_seq / 4;
+    // flattened unit offsets: exclusive prefix sum of units per sequence
     int64_t mine = 0;
-    for (int b = b0; b < b1; ++b) mine += tiles_of(seqlens[b]);
+    for (int b = b0; b < b1; ++b) mine += units_of(seqlens[b], unit_rows);
     int64_t total;
     int64_t f = block_exclusive_scan(mine, scan_smem, &total);
     const int used = used_ctas(total, ctas);
-    // splits per sequence (the consecutive CTAs its tiles fall on)
+    // splits per sequence (the consecutive CTAs its units fall on)
     int64_t split_slots = 0;
     for (int b = b0; b < b1; ++b) {
-        const int64_t t0 = f, t1 = f + tiles_of(seqlens[b]);
+        const int64_t t0 = f, t1 = f + units_of(seqlens[b], unit_rows);
         int first = -1, nsplit = 0;
         if (t1 > t0) {
             first = cta_of(total, used, t0);
@@ -91,22 +94,59 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t *__res
         seq_info[4 * b + 3] = (int32_t)sl;
         if (seq_info[4 * b + 2] >= 2) sl += seq_info[4 * b + 2];
     }
-    for (int c = threadIdx.x; c < ctas; c += kPlanThreads) {
+    for (int c = threadIdx.x; c < ctas; c += blockDim.x) {
         ranges[2 * c] = (int32_t)cta_begin(total, used, c);
         ranges[2 * c + 1] = (int32_t)cta_begin(total, used, c + 1);
-        if (c >= used) cta_seq[c] = batch;  // no tiles
+        if (c >= used) cta_seq[c] = batch;  // no units
     }
-    for (int i = threadIdx.x; i < 2 * batch * groups; i += kPlanThreads) counters[i] = 0;
+    for (int i = threadIdx.x; i < 2 * batch * groups; i += blockDim.x) counters[i] = 0;
     if (threadIdx.x == 0) {
         tile_off[batch] = (int32_t)total;
+        ws[hdr + kSchCtas] = ctas;
+        ws[hdr + kSchGroups] = groups;
+        ws[hdr + kSchTotal] = (int32_t)total;
+        ws[hdr + kSchSlotsUsed] = (int32_t)slots;
+        ws[hdr + kSchGroupCols] = gcols;
+        ws[hdr + kSchMode] = mode;
+    }
+}
+
+// One CTA of kPlanThreads threads: the pair schedule and, for more than 16 query columns, the duo
+// schedule (whose column-group width depends on the shortest nonempty sequence).  Writes the header
+// (and clears the status word) so that the decode kernels can check that they run on a plan for
+// their own grid.
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t *__restrict__ seqlens, int batch, int ncols,
+                                                            int num_sms, int32_t *__restrict__ ws, WsLayout lay) {
+    // Launched as a programmatic dependent: nothing is read (seqlens may come from the
+    // preceding kernel) or written (that kernel may still read the workspace) before it
+    // completes.  Then the decode kernel may start its prologue: it waits for this grid in
+    // turn before reading the workspace.  Both are no-ops without programmatic launch.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ int64_t scan_smem[32];
+    __shared__ int min_smem[32];
+    const int per = (batch + kPlanThreads - 1) / kPlanThreads;
+    const int b0 = min(batch, (int)threadIdx.x * per), b1 = min(batch, b0 + per);
+    plan_schedule(seqlens, batch, b0, b1, lay.ctas, lay.groups, kTileRows, group_cols(ncols), 0, ws, lay.pair,
+                  kHdrPair, scan_smem);
+    if (lay.has_duo) {
+        int mn = 0x7fffffff;
+        for (int b = b0; b < b1; ++b) {
+            const int L = seqlens[b];
+            if (L > 0) mn = min(mn, L);
+        }
+        mn = block_min(mn, min_smem);
+        const int mode = duo_mode(ncols, mn == 0x7fffffff ? 0 : mn);
+        const int groups = duo_groups(ncols, mode);
+        plan_schedule(seqlens, batch, b0, b1, num_ctas(num_sms, groups), groups, kDuoRows, duo_group_cols(mode), mode,
+                      ws, lay.duo, kHdrDuo, scan_smem);
+    }
+    if (threadIdx.x == 0) {
         ws[kHdrStatus] = 0;
-        ws[kHdrCtas] = ctas;
-        ws[kHdrGroups] = groups;
         ws[kHdrBatch] = batch;
-        ws[kHdrTotalTiles] = (int32_t)total;
         ws[kHdrCols] = ncols;
-        ws[kHdrSlotsUsed] = (int32_t)slots;
         ws[kHdrSlotsMax] = lay.slots;
+        ws[kHdrSchedUsed] = 0;
     }
 }
 
@@ -116,7 +156,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const int32_t *__restrict_
                                                       const float *__restrict__ lsepart, int ncols, WsLayout lay,
                                                       __nv_bfloat16 *__restrict__ o, float *__restrict__ lse) {
     const int n = blockIdx.x, b = blockIdx.y;
-    const int32_t *seq_info = ws + lay.seq_info / 4;
+    // the schedule of the decode that wrote the partials
+    const int32_t *seq_info = ws + (ws[kHdrSchedUsed] == 1 ? lay.duo.seq_info : lay.pair.seq_info) / 4;
     const int nsplit = seq_info[4 * b + 2];
     if (nsplit == 1) return;  // written by the decode kernel
     const int64_t orow = ((int64_t)b * ncols + n) * kDv + 4 * threadIdx.x;

@@ -246,35 +246,66 @@ def _a256(x):
     return (x + 255) & ~255
 
 
+def _sched_offsets(off, batch, ctas_max, groups_max):
+    """Byte offsets of one schedule's tables in the workspace (the layout of plan_core.h)."""
+    t = {"ranges": off}
+    off += _a256(4 * 2 * ctas_max)
+    t["seq"] = off
+    off += _a256(4 * ctas_max)
+    t["tile"] = off
+    off += _a256(4 * (batch + 1))
+    t["info"] = off
+    off += _a256(4 * 4 * batch)
+    t["counters"] = off
+    off += _a256(4 * 2 * batch * groups_max)
+    return t, off
+
+
 @pytest.mark.parametrize("batch", [1, 7, 1024, 1500, 5000])
-def test_device_plan_matches_host_plan(batch):
-    """The block-scan plan kernel writes the same schedule as the host mirror (ranges, per-
-    sequence tiles / first unit / splits / slot offsets, tile offsets), for batches that give
-    each plan thread zero, one or several sequences, with empty sequences mixed in."""
+@pytest.mark.parametrize("heads", [16, 128])
+def test_device_plan_matches_host_plan(batch, heads):
+    """The block-scan plan kernel writes the same schedules as the host mirror (ranges, per-
+    sequence units / first unit / splits / slot offsets, unit offsets, the grouping the M = 256
+    kernel takes), for batches that give each plan thread zero, one or several sequences, with
+    empty sequences mixed in."""
     from mla_decode_attention_etap_b200 import MlaDecoder, mla_decode_plan_host
-    rng = np.random.default_rng(batch)
+    rng = np.random.default_rng(batch + heads)
     lens = rng.integers(0, 3000, size=batch).astype(np.int32)
     lens[rng.random(batch) < 0.2] = 0
+    if heads == 128 and batch % 2:  # every nonempty sequence long: one 128-column group
+        lens = np.where(lens > 0, lens + 8192, 0).astype(np.int32)
     dev = torch.device("cuda")
-    dec = MlaDecoder(batch, 1, 16, device=dev)
+    dec = MlaDecoder(batch, 1, heads, device=dev)
     dec.plan(torch.tensor(lens, device=dev))
     torch.cuda.synchronize()
-    ranges, info, nct, _ = mla_decode_plan_host(lens, 1, 16, dec.n_sms)
     ws = dec.workspace.view(torch.int32).cpu().numpy()
-    off_ranges = _a256(4 * 64)
-    off_seq = off_ranges + _a256(4 * 2 * nct)
-    off_tile = off_seq + _a256(4 * nct)
-    off_info = off_tile + _a256(4 * (batch + 1))
-    np.testing.assert_array_equal(ws[off_ranges // 4: off_ranges // 4 + 2 * nct].reshape(-1, 2), ranges)
-    np.testing.assert_array_equal(ws[off_info // 4: off_info // 4 + 4 * batch].reshape(-1, 4), info)
-    tiles = (lens.astype(np.int64) + 127) // 128
-    tile_off = np.concatenate([[0], np.cumsum(tiles)]).astype(np.int64)
-    np.testing.assert_array_equal(ws[off_tile // 4: off_tile // 4 + batch + 1], tile_off.astype(np.int32))
-    # each unit's first sequence: the one whose tile range holds the unit's first tile (batch if none)
-    want = np.array([int(np.searchsorted(tile_off, fb, side="right") - 1) if fb < fe else batch
-                     for fb, fe in ranges], dtype=np.int32)
-    np.testing.assert_array_equal(ws[off_seq // 4: off_seq // 4 + nct], want)
-    assert ws[0] == 0 and ws[1] == nct and ws[3] == batch and ws[4] == int(tiles.sum())
+    ncols = heads
+    n_sms = dec.n_sms
+    # sizing of the two schedules (plan_core.h ws_layout)
+    pair_groups = 1 if ncols <= 16 else (ncols + 31) // 32
+    pair_ctas = max(1, n_sms // 2 // pair_groups)
+    tabs = {}
+    tabs[0], off = _sched_offsets(_a256(4 * 64), batch, pair_ctas, pair_groups)
+    if ncols > 16:
+        g0 = (ncols + 63) // 64
+        c_max = max(1, n_sms // 2 // ((ncols + 127) // 128 if ncols > 64 else g0))
+        tabs[1], off = _sched_offsets(off, batch, c_max, g0)
+    for schedule, hdr in ((0, 8), (1, 16)):
+        if schedule == 1 and ncols <= 16:
+            continue
+        ranges, info, nct, ngr, rows, gcols = mla_decode_plan_host(lens, 1, heads, n_sms, schedule)
+        t = tabs[schedule]
+        np.testing.assert_array_equal(ws[t["ranges"] // 4: t["ranges"] // 4 + 2 * nct].reshape(-1, 2), ranges)
+        np.testing.assert_array_equal(ws[t["info"] // 4: t["info"] // 4 + 4 * batch].reshape(-1, 4), info)
+        units = (lens.astype(np.int64) + rows - 1) // rows
+        tile_off = np.concatenate([[0], np.cumsum(units)]).astype(np.int64)
+        np.testing.assert_array_equal(ws[t["tile"] // 4: t["tile"] // 4 + batch + 1], tile_off.astype(np.int32))
+        # each unit's first sequence: the one whose range holds the unit's first tile (batch if none)
+        want = np.array([int(np.searchsorted(tile_off, fb, side="right") - 1) if fb < fe else batch
+                         for fb, fe in ranges], dtype=np.int32)
+        np.testing.assert_array_equal(ws[t["seq"] // 4: t["seq"] // 4 + nct], want)
+        assert ws[hdr] == nct and ws[hdr + 1] == ngr and ws[hdr + 2] == int(units.sum()) and ws[hdr + 4] == gcols
+    assert ws[0] == 0 and ws[1] == batch and ws[2] == ncols
 
 
 @pytest.mark.parametrize("heads,q_len,causal", [(64, 1, False), (128, 2, False), (32, 4, True), (16, 8, True),
