@@ -225,13 +225,13 @@ TRACE_ROLES = ("K-tile producer", "step-1 issuer", "value producer", "softmax", 
 def mla_decode_fwd_trace(q, kv, seqlens, block_table, softmax_scale, causal, o, lse, workspace, n_sms, trace,
                          stream=None) -> None:
     """mla_decode_fwd that also records the event stamps of cluster 0's roles into ``trace`` (int64 device
-    tensor of 2 * 5 * cap + 8 * n_sms elements, zeroed by the caller, made by trace_buffer()); see
+    tensor of 2 * 5 * cap + 4 * n_sms elements, zeroed by the caller, made by trace_buffer()); see
     decode_trace_events() and decode_trace_spans()."""
     _require_cuda(q, "q")
     check_decode_args(q, kv, seqlens, block_table, o, lse, workspace)
     _require(trace, "trace", torch.int64, q.device, dim=1)
-    cap = (trace.numel() - 8 * n_sms) // (2 * len(TRACE_ROLES))
-    if cap < 1 or trace.numel() != 2 * len(TRACE_ROLES) * cap + 8 * n_sms:
+    cap = (trace.numel() - 4 * n_sms) // (2 * len(TRACE_ROLES))
+    if cap < 1 or trace.numel() != 2 * len(TRACE_ROLES) * cap + 4 * n_sms:
         raise ValueError("trace: use trace_buffer(cap, n_sms)")
     B, q_len, h, _ = q.shape
     if block_table is not None:
@@ -246,7 +246,7 @@ def mla_decode_fwd_trace(q, kv, seqlens, block_table, softmax_scale, causal, o, 
 
 def trace_buffer(cap: int, n_sms: int, device=None):
     """A zeroed trace buffer for mla_decode_fwd_trace: [2 CTAs][5 roles][cap] stamps, then [n_sms][4]."""
-    return torch.zeros(2 * len(TRACE_ROLES) * cap + 8 * n_sms, dtype=torch.int64, device=device)
+    return torch.zeros(2 * len(TRACE_ROLES) * cap + 4 * n_sms, dtype=torch.int64, device=device)
 
 
 def decode_trace_spans(trace, n_sms: int):
@@ -254,7 +254,7 @@ def decode_trace_spans(trace, n_sms: int):
     earliest entry (rows of CTAs that did not run stay 0)."""
     import numpy as np
     t = np.asarray(trace.cpu() if isinstance(trace, torch.Tensor) else trace).astype(np.int64)
-    sp = t[len(t) - 8 * n_sms:].reshape(n_sms, 8).copy()
+    sp = t[len(t) - 4 * n_sms:].reshape(n_sms, 4).copy()
     live = sp[:, 0] > 0
     if live.any():
         sp[live] -= sp[live, 0].min()
@@ -266,7 +266,7 @@ def decode_trace_events(trace, n_sms: int = None):
     import numpy as np
     t = np.asarray(trace.cpu() if isinstance(trace, torch.Tensor) else trace).astype(np.uint64)
     if n_sms is not None:
-        t = t[:len(t) - 8 * n_sms]
+        t = t[:len(t) - 4 * n_sms]
     t = t.reshape(2, len(TRACE_ROLES), -1)
     out = []
     for cta in range(t.shape[0]):

@@ -213,30 +213,6 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
             bool ok = true;
             TraceRow tr;
             tr.init(p, 0);
-            // L2 prefetch of this CTA's rows of the next unit, so that its loads hit L2
-            TileCursor ahead;
-            ahead.init(tile_off, seq0, fb, fe);
-            auto prefetch = [&]() {
-                if (!ahead.valid) return;
-                const int bp = ahead.b;
-                int Lp = p.seqlens[bp];
-                if ((int64_t)Lp > l_cap) Lp = (int)l_cap;
-                const int r0 = ahead.t * kDuoRows + kTileRows * (int)rank;
-                for (int hh = 0; hh < 2; ++hh) {
-                    if (Lp - r0 <= 64 * hh) break;
-                    int yp;
-                    if (p.paged) {
-                        const int blk = p.block_table[(int64_t)bp * p.max_blocks + (r0 >> 6) + hh];
-                        if (blk < 0 || (int64_t)blk * kPage >= p.kv_rows) continue;
-                        yp = blk * kPage;
-                    } else {
-                        yp = (int)((int64_t)bp * p.kv_rows + r0 + 64 * hh);
-                    }
-                    for (int c = 0; c < 9; ++c) tma_prefetch_l2_2d(&tm.kv, 64 * c, yp);
-                }
-                ahead.advance(tile_off);
-            };
-            prefetch();
             SegIter it;
             it.init_at(seq0, fb, fe);
             int b, t0, t1, seg = 0;
@@ -253,7 +229,6 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
                     tr.put(kEvQ, seg);
                 }
                 for (int tp = t0; tp < t1 && ok; ++tp) {
-                    prefetch();
                     int y[2];
                     bool loaded[2];
                     locate(b, tp * kDuoRows + kTileRows * (int)rank, L, y, loaded);
@@ -273,6 +248,11 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
                 }
                 ++seg;
             }
+            // Tail: the last releases of the slots and of Q arrive by multicast commit; wait for them
+            // so that nothing lands in this CTA's shared memory after it leaves.
+            for (uint32_t g = g1; ok && g < g1 + C::NS1; ++g)
+                ok = poll_phase(bar(BR::S1E + g % C::NS1), ((g / C::NS1) & 1) ^ 1, wc, status);
+            if (ok && seg > 0) ok = poll_phase(bar(BR::QE), (seg - 1) & 1, wc, status);
         }
         __syncwarp();
     } else if (warp == 2) {
@@ -344,6 +324,11 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
                     }
                 }
             }
+            // Tail: the last slot releases (multicast commits) land before this CTA leaves.
+            for (uint32_t g = g3; ok && g < g3 + C::NS3; ++g) {
+                if (lane == 0) ok = poll_phase(bar(BR::S3E + g % C::NS3), ((g / C::NS3) & 1) ^ 1, wc, status);
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            }
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -412,6 +397,10 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
                     break;
                 }
             }
+            // Tail: both CTAs' last releases of the score buffers (the odd CTA's arrive is remote)
+            // land before this CTA leaves.
+            for (int k = kq; k < kq + 2 && !wc->abort; ++k)
+                if (!poll_phase(bar(BR::SE + (k & 1)), ((k >> 1) & 1) ^ 1, wc, status)) break;
             pv_pending = true;  // FINAL is committed (and drained) at the end of the kernel
         }
         __syncwarp();
@@ -1024,7 +1013,7 @@ __global__ void __launch_bounds__(kDuoThreads, 1)
     volatile WaitCtl *wc = reinterpret_cast<volatile WaitCtl *>(smem + kDuoCtlMisc + 16);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kDuoCtlMisc);
     // trace: every CTA's entry, start of work (after the plan), end of work and exit
-    unsigned long long *span = p.trace ? p.trace + (size_t)2 * kTraceRoles * p.trace_cap + 8 * (size_t)blockIdx.x : nullptr;
+    unsigned long long *span = p.trace ? p.trace + (size_t)2 * kTraceRoles * p.trace_cap + 4 * (size_t)blockIdx.x : nullptr;
     if (span && threadIdx.x == 0) span[0] = global_timer_ns();
 
     if (threadIdx.x == 0) {
@@ -1103,9 +1092,12 @@ __global__ void __launch_bounds__(kDuoThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (span && threadIdx.x == 0) span[2] = global_timer_ns();
-    cluster_sync();  // no CTA leaves while its peer may still write into its shared memory
-    if (span && threadIdx.x == 0) span[4] = global_timer_ns();  // DEBUG
-    if (span && threadIdx.x == 32) span[5] = global_timer_ns();  // DEBUG
+    // No CTA leaves while its peer may still write into its shared memory.  Every operation that
+    // targets a CTA's shared memory (TMA bytes, st.async, remote and multicast arrivals) has been
+    // waited for by that CTA above (the producers' tails included), so the barrier needs no
+    // ordering of its own: a releasing arrive would wait for every global store of the CTA, tens
+    // of microseconds while the memory system is busy.
+    cluster_sync_relaxed_arrive();
     if (wc->abort) {
         // After an abort a peer's last st.async or bulk copy may not have been waited for: let it
         // land before either CTA leaves (no thread sends after the barrier above).
@@ -1113,11 +1105,10 @@ __global__ void __launch_bounds__(kDuoThreads, 1)
         while (global_timer_ns() - t_q < 20000ull) {
         }
     }
-    cluster_sync();
-    if (span && threadIdx.x == 32) span[6] = global_timer_ns();  // DEBUG
+    cluster_sync_relaxed_arrive();
     tc_fence_after();
     if (warp == 1) tmem_dealloc_pair(tmem, 512);
-    if (span && threadIdx.x == 32) span[3] = global_timer_ns() | (wc->abort ? (1ull << 62) : 0ull);  // DEBUG
+    if (span && threadIdx.x == 32) span[3] = global_timer_ns();
 }
 
 }  // namespace mla

@@ -16,7 +16,7 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t)::"memory");  // not moved across memory operations
     return t;
 }
 
@@ -123,6 +123,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t remote_bar
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
+// Cluster barrier whose arrive carries no ordering of its own: the caller orders what must be
+// visible before it (a fence by one thread after a CTA barrier, which is cumulative).
+__device__ __forceinline__ void cluster_sync_relaxed_arrive() {
+    asm volatile("barrier.cluster.arrive.relaxed;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
