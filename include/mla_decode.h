@@ -101,11 +101,15 @@ MLA_API int mla_decode_plan(const int32_t *seqlens, int batch, int q_len, int nu
 /*
  * The decode itself (ETAP steps 1-4 of the pages, plus the split-KV partial
  * outputs and, unless MLA_FLAG_SKIP_COMBINE is set, their merge).  Without that
- * flag the merge runs inside the decode kernel: the last CTA to finish a split
- * of a sequence merges all of its splits (same arithmetic as mla_combine, so the
+ * flag the merge is part of the call, with the arithmetic of mla_combine (so the
  * results are bitwise equal), and sequences with L_b = 0 get O = 0, LSE = -inf.
- * (When num_sms allows more splits per sequence than the kernel's merge buffer
- * holds, fwd launches the combine kernel after the decode instead.)
+ * With 16 query columns or fewer (and for mla_decode_fwd_fp8) the last CTA to
+ * finish a split of a sequence merges all of its splits inside the decode kernel
+ * (when num_sms allows more splits per sequence than that merge's buffer holds,
+ * the combine kernel runs after the decode instead).  With more columns on the
+ * bf16 cache the combine kernel is launched behind the decode and starts on the
+ * SMs the decode leaves: each of its CTAs waits for the split counters of its
+ * own sequence, so early sequences are merged while the decode still runs.
  *   q            bf16 [batch, q_len, num_heads, 576], 16-byte aligned
  *   kv           contiguous: bf16 [batch, kv_rows, 576];
  *                paged (block_table != NULL): bf16 [kv_rows / 64, 64, 576], i.e. kv_rows = num_blocks*64
@@ -178,8 +182,10 @@ MLA_API int mla_decode_fwd_fp8(const void *q, const void *kv8, const float *kv_s
  * workspace: lse = ln sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s, for
  * every sequence split over several CTAs; also writes O = 0, LSE = -inf for
  * empty sequences. Sequences handled by one CTA were already written by fwd.
+ * Runs after everything before it on the stream.  It also rearms the split
+ * counters in the workspace, which is why the workspace is writable here.
  */
-MLA_API int mla_combine(const void *workspace, int batch, int q_len, int num_heads, int num_sms,
+MLA_API int mla_combine(void *workspace, int batch, int q_len, int num_heads, int num_sms,
                 void *o, float *lse, void *stream);
 
 /*

@@ -60,6 +60,7 @@ struct DecodeParams {
     int32_t *counters;  // [batch][groups][2]: split CTAs done per (sequence, column group, rank)
     int slots;          // partial slots (stride between the two ranks' LSE partial arrays)
     int fuse_merge;     // the last split CTA of a sequence merges the partials (no combine launch)
+    int signal_combine; // count stored split partials for the combine kernel that follows
     unsigned long long *trace;  // measurement: event stamps of cluster 0's roles, or NULL
     int trace_cap;              // stamps per (CTA, role) in `trace`
 };

@@ -37,13 +37,12 @@
 #pragma once
 
 #include "etap_common.cuh"
-#include "merge.cuh"
 
 namespace mla {
 
 // Shared-memory control block (identical in both configurations, so that one prologue serves both).
 constexpr uint32_t kDuoCtlBar = 0;        // mbarriers
-constexpr uint32_t kDuoCtlMisc = 512;     // +0 TMEM address, +16 WaitCtl, +48 merge flag, +64 received votes (2 x 16 B)
+constexpr uint32_t kDuoCtlMisc = 512;     // +0 TMEM address, +16 WaitCtl, +64 received votes (2 x 16 B)
 constexpr uint32_t kDuoCtlM = 1024;       // float[128] running maximum per column (log2 units)
 constexpr uint32_t kDuoCtlAlpha = 1536;   // float[128] rescale factor of the current tile pair
 constexpr uint32_t kDuoCtlRed = 2048;     // float[4][128] per-quadrant partial maxima / sums
@@ -51,9 +50,7 @@ constexpr uint32_t kDuoCtlMx = 4096;      // float[128] peer's tile maxima (rece
 constexpr uint32_t kDuoCtlLx = 4608;      // float[128] peer's row sums (received)
 constexpr uint32_t kDuoCtlMt = 5120;      // float[128] this CTA's tile maxima / row sums
 constexpr uint32_t kDuoCtlVis = 5632;     // int[128] visible rows per column of the current sequence
-constexpr uint32_t kDuoCtlStage = 6144;   // float[1024]: the split merge's partial LSEs and merged LSEs
-constexpr int kDuoStageFloats = 1024;
-constexpr uint32_t kDuoCtlEnd = 10240;    // data regions start here (1024-aligned)
+constexpr uint32_t kDuoCtlEnd = 6144;     // data regions start here (1024-aligned)
 constexpr int kDuoThreads = 384;
 
 // NC query columns per cluster, P as hi + lo (SPLIT), NS1 K-chunk slots, NS3 value-pair slots.
@@ -88,7 +85,7 @@ constexpr uint32_t kDuoSmemAlloc =
 
 template <class C>
 constexpr bool duo_cfg_fits() {
-    return C::BYTES + 1024 <= 232448 && kDuoCtlStage + 4 * kDuoStageFloats <= kDuoCtlEnd && C::S_COL + 2 * C::NC <= 512 && C::P_PITCH == 128 && C::NS1 <= 3 &&
+    return C::BYTES + 1024 <= 232448 && kDuoCtlVis + 512 <= kDuoCtlEnd && C::S_COL + 2 * C::NC <= 512 && C::P_PITCH == 128 && C::NS1 <= 3 &&
            C::NS3 <= 3 && C::OFF_Q % 1024 == 0 && C::OFF_P % 1024 == 0 && C::NC <= 128 && C::NH % 16 == 0;
 }
 static_assert(duo_cfg_fits<DuoCfg64>() && duo_cfg_fits<DuoCfg128>(), "shared memory / TMEM plan");
@@ -131,8 +128,7 @@ enum : int {
     kEvSmEpiDone = 37,  // softmax: epilogue ends
     kEvEpiS3 = 38,      // epilogue: the segment's last step 3 observed complete
     kEvEpiL = 39,       // epilogue: column sums of both CTAs known
-    kEvEpiO = 40,       // epilogue: outputs (or partials) stored
-    kEvMerge = 41       // epilogue: this CTA merges the sequence's splits (index: splits)
+    kEvEpiO = 40        // epilogue: outputs (or partials) stored
 };
 
 template <class C>
@@ -866,130 +862,16 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
                             p.lsepart[((int64_t)rank * p.slots + slot) * p.ncols + ng] = lse;
                     }
                 }
-                if (nsplit >= 2 && rank == 1 && tid < NC) {
-                    // rank 1's partial LSEs (equal to rank 0's) for the separate combine's row of rank 1
-                    const int ng = grp * NC + tid;
-                    if (ng < p.ncols) {
-                        const float l = col_l(tid);
-                        const bool empty = !(l > 0.f) || m_s[tid] == -INFINITY;
-                        p.lsepart[((int64_t)rank * p.slots + slot) * p.ncols + ng] =
-                            empty ? -INFINITY : (m_s[tid] + __log2f(l)) * 0.69314718055994531f;
-                    }
-                }
                 tr.put(kEvEpiO, nsplit);
-                if (nsplit >= 2 && p.fuse_merge) {
-                    // Split-KV merge in the kernel: the last CTA (of this rank) to finish a split of
-                    // sequence b merges all splits for its 256 latent rows and this column group.
+                if (nsplit >= 2 && p.signal_combine) {
+                    // this CTA's partial of the split is stored: count it for the combine kernel
+                    // (release: the CTA barrier and one thread's release add cover every thread's
+                    // stores)
                     named_bar_sync(SMX, NSM);
-                    volatile int *merge_flag = reinterpret_cast<volatile int *>(smem + kDuoCtlMisc + 48);
-                    int32_t *cnt = p.counters + ((int64_t)b * groups + grp) * 2 + rank;
-                    if (tid == 0) {
-                        __threadfence();
-                        const bool last = atomicAdd(cnt, 1) == nsplit - 1;
-                        if (last) __threadfence();
-                        *merge_flag = last;
-                    }
-                    named_bar_sync(SMX, NSM);
-                    if (*merge_flag) {
-                        tr.put(kEvMerge, nsplit);
-                        // Passes of MP columns (all NC when the partial LSEs of every split fit in the staging
-                        // area): the partial LSEs are staged with one parallel load, merged per column in split
-                        // order, and each thread accumulates 4 consecutive latent rows x MP/4 columns, 8
-                        // columns x 2 splits of loads in flight.  The arithmetic and its order are those of the
-                        // combine kernel, so both give identical bits.
-                        const int s0 = seq_info[4 * b + 3];
-                        int MP = NC;
-                        while (MP > 8 && (nsplit + 1) * MP > kDuoStageFloats) MP >>= 1;
-                        float *ls = reinterpret_cast<float *>(smem + kDuoCtlStage);  // [nsplit][MP]
-                        float *lt = ls + nsplit * MP;                               // [MP]
-                        const int d4 = 256 * (int)rank + 4 * (tid & 63);
-                        const int cpt = MP / 4;                                     // columns per thread
-                        const int cq = (tid >> 6) * cpt;
-                        for (int cp = 0; cp < NC; cp += MP) {
-                            const int cbase = grp * NC + cp;
-                            const int nn = p.ncols - cbase < MP ? p.ncols - cbase : MP;
-                            if (nn <= 0) break;
-                            const float *lsrc = p.lsepart + ((int64_t)rank * p.slots + s0) * p.ncols + cbase;
-                            for (int i = tid; i < nsplit * MP; i += NSM) {
-                                const int sp = i / MP, n = i - sp * MP;
-                                ls[i] = n < nn ? __ldcg(lsrc + (int64_t)sp * p.ncols + n) : -INFINITY;
-                            }
-                            named_bar_sync(SMX, NSM);
-                            if (tid < MP) lt[tid] = merged_lse([&](int sp) { return ls[sp * MP + tid]; }, nsplit);
-                            named_bar_sync(SMX, NSM);
-#pragma unroll 1
-                            for (int c0 = 0; c0 < cpt; c0 += 8) {
-                                float acc[8][4];
-#pragma unroll
-                                for (int jj = 0; jj < 8; ++jj) acc[jj][0] = acc[jj][1] = acc[jj][2] = acc[jj][3] = 0.f;
-                                // column of slot jj: clamped to a real column for the load, weight 0 past nn
-                                auto colof = [&](int jj) { const int c = cq + c0 + jj; return c < nn ? c : nn - 1; };
-                                const float *op = p.opart + ((int64_t)s0 * p.ncols + cbase) * kDv + d4;
-                                auto accum = [&](int sp, const float4 (&v)[8]) {
-#pragma unroll
-                                    for (int jj = 0; jj < 8; ++jj) {
-                                        const int c = cq + c0 + jj;
-                                        const float lv = c < nn ? lt[c] : -INFINITY;
-                                        if (lv != -INFINITY) {
-                                            const float w = merge_weight(ls[sp * MP + c], lv);
-                                            acc[jj][0] = fmaf(w, v[jj].x, acc[jj][0]);
-                                            acc[jj][1] = fmaf(w, v[jj].y, acc[jj][1]);
-                                            acc[jj][2] = fmaf(w, v[jj].z, acc[jj][2]);
-                                            acc[jj][3] = fmaf(w, v[jj].w, acc[jj][3]);
-                                        }
-                                    }
-                                };
-                                int sp = 0;
-#pragma unroll 1
-                                for (; sp + 1 < nsplit; sp += 2) {
-                                    float4 va[8], vb[8];
-#pragma unroll
-                                    for (int jj = 0; jj < 8; ++jj) {
-                                        va[jj] = __ldcg(reinterpret_cast<const float4 *>(op + ((int64_t)sp * p.ncols + colof(jj)) * kDv));
-                                        vb[jj] = __ldcg(reinterpret_cast<const float4 *>(op + ((int64_t)(sp + 1) * p.ncols + colof(jj)) * kDv));
-                                    }
-                                    accum(sp, va);
-                                    accum(sp + 1, vb);
-                                }
-                                if (sp < nsplit) {
-                                    float4 va[8];
-#pragma unroll
-                                    for (int jj = 0; jj < 8; ++jj)
-                                        va[jj] = __ldcg(reinterpret_cast<const float4 *>(op + ((int64_t)sp * p.ncols + colof(jj)) * kDv));
-                                    accum(sp, va);
-                                }
-#pragma unroll
-                                for (int jj = 0; jj < 8; ++jj) {
-                                    const int c = cq + c0 + jj;
-                                    if (c >= nn) break;
-                                    const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc[jj][0], acc[jj][1]);
-                                    const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc[jj][2], acc[jj][3]);
-                                    uint2 packed;
-                                    packed.x = *reinterpret_cast<const uint32_t *>(&lo2);
-                                    packed.y = *reinterpret_cast<const uint32_t *>(&hi2);
-                                    *reinterpret_cast<uint2 *>(p.o + ((int64_t)b * p.ncols + cbase + c) * kDv + d4) = packed;
-                                    if (rank == 0 && (tid & 63) == 0) p.lse[(int64_t)b * p.ncols + cbase + c] = lt[c];
-                                }
-                            }
-                            named_bar_sync(SMX, NSM);  // ls / lt are rewritten by the next pass
-                        }
-                        if (tid == 0) *cnt = 0;  // ready for the next call
-                    }
+                    if (tid == 0) red_add_release_gpu(p.counters + ((int64_t)b * groups + grp) * 2 + rank, 1);
                 }
                 tr.put(kEvSmEpiDone, kl);
                 tc_fence_before();
-            }
-        }
-        if (p.fuse_merge && !stop && ok) {
-            // Sequences without a single KV row get no split: O = 0 and LSE = -inf, written by
-            // cluster b mod (number of clusters), each CTA for its 256 latent rows.
-            const int ncl = (int)(gridDim.x >> 1);
-            const int d = 256 * (int)rank + tid;
-            for (int bb = (int)(blockIdx.x >> 1); bb < p.batch; bb += ncl) {
-                if (seq_info[4 * bb + 2] != 0) continue;
-                for (int n = 0; n < p.ncols; ++n) p.o[((int64_t)bb * p.ncols + n) * kDv + d] = __float2bfloat16_rn(0.f);
-                if (rank == 0 && sw == 0)
-                    for (int n = lane; n < p.ncols; n += 32) p.lse[(int64_t)bb * p.ncols + n] = -INFINITY;
             }
         }
         if (stop || !ok) wc->abort = 1;

@@ -157,6 +157,34 @@ cudaError_t launch_duo(const mla::DuoMaps &maps, const mla::DecodeParams &p, int
     return cudaLaunchKernelEx(&cfg, mla::etap_duo_kernel<mla::DuoCfg64, mla::DuoCfg128>, maps, p);
 }
 
+// The combine kernel, launched as a programmatic dependent of what precedes it on the stream:
+// with spin = 0 it waits for that whole grid; with spin = 1 (after the duo kernel only) its CTAs
+// wait for their own sequence's split counters.
+int launch_combine(void *workspace, int batch, int q_len, int num_heads, int num_sms, void *o, float *lse, int spin,
+                   unsigned long long wait_limit_ns, cudaStream_t s) {
+    const mla::WsLayout lay = mla::ws_layout(batch, q_len, num_heads, num_sms);
+    const int ncols = q_len * num_heads;
+    char *ws = reinterpret_cast<char *>(workspace);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ncols, batch, 1);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, mla::combine_kernel, reinterpret_cast<int32_t *>(ws),
+                                       reinterpret_cast<const float *>(ws + lay.opart),
+                                       reinterpret_cast<const float *>(ws + lay.lsepart), ncols, lay,
+                                       reinterpret_cast<__nv_bfloat16 *>(o), lse, spin, wait_limit_ns);
+    if (e != cudaSuccess) return cuda_fail(e, "combine_kernel launch");
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "combine_kernel launch");
+    return MLA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -265,22 +293,14 @@ int mla_decode_plan(const int32_t *seqlens, int batch, int q_len, int num_heads,
     return MLA_OK;
 }
 
-int mla_combine(const void *workspace, int batch, int q_len, int num_heads, int num_sms, void *o, float *lse,
+int mla_combine(void *workspace, int batch, int q_len, int num_heads, int num_sms, void *o, float *lse,
                 void *stream) {
     int st = check_shape(batch, q_len, num_heads, num_sms);
     if (st != MLA_OK) return st;
     if (!workspace || !o || !lse) return MLA_ERR_INVALID_ARG;
     if (!aligned(workspace, 256) || !aligned(o, 16) || !aligned(lse, 4)) return MLA_ERR_ALIGNMENT;
-    const mla::WsLayout lay = mla::ws_layout(batch, q_len, num_heads, num_sms);
-    const int ncols = q_len * num_heads;
-    const char *ws = reinterpret_cast<const char *>(workspace);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    mla::combine_kernel<<<dim3(ncols, batch), 128, 0, s>>>(
-        reinterpret_cast<const int32_t *>(ws), reinterpret_cast<const float *>(ws + lay.opart),
-        reinterpret_cast<const float *>(ws + lay.lsepart), ncols, lay, reinterpret_cast<__nv_bfloat16 *>(o), lse);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "combine_kernel launch");
-    return MLA_OK;
+    return launch_combine(workspace, batch, q_len, num_heads, num_sms, o, lse, 0, mla::kWaitLimitNs,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 int mla_decode_fwd(const void *q, const void *kv, const int32_t *seqlens, const int32_t *block_table, int batch,
@@ -410,7 +430,10 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
         p.seq_info_off = (int)(lay.duo.seq_info / 4);
         p.cta_seq_off = (int)(lay.duo.cta_seq / 4);
         p.counters = reinterpret_cast<int32_t *>(ws + lay.duo.counters);
-        p.fuse_merge = (flags & MLA_FLAG_SKIP_COMBINE) ? 0 : 1;
+        // The splits are merged by the combine kernel: spread over all SMs it costs less than the
+        // in-kernel merge of the pair kernel, which would fall on the last split's CTA pair.
+        p.fuse_merge = 0;
+        p.signal_combine = (flags & MLA_FLAG_SKIP_COMBINE) ? 0 : 1;
         int clusters = 0;
         for (int mode = 0; mode < 2; ++mode) {
             if (mode == 1 && !mla::duo_mode1_possible(ncols)) break;
@@ -421,7 +444,8 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
         if (e != cudaSuccess) return cuda_fail(e, "etap_duo_kernel launch");
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "etap_duo_kernel launch");
-        return MLA_OK;
+        if (flags & MLA_FLAG_SKIP_COMBINE) return MLA_OK;
+        return launch_combine(workspace, batch, q_len, num_heads, num_sms, o, lse, 1, p.wait_limit_ns, s);
     }
     const int clusters = lay.ctas * lay.groups;
     if (fp8)

@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "etap_common.cuh"
 #include "merge.cuh"
 #include "plan_core.h"
 
@@ -100,6 +101,7 @@ __device__ void plan_schedule(const int32_t *__restrict__ seqlens, int batch, in
         if (c >= used) cta_seq[c] = batch;  // no units
     }
     for (int i = threadIdx.x; i < 2 * batch * groups; i += blockDim.x) counters[i] = 0;
+    for (int i = threadIdx.x; i < batch; i += blockDim.x) ws[sc.done / 4 + i] = 0;
     if (threadIdx.x == 0) {
         tile_off[batch] = (int32_t)total;
         ws[hdr + kSchCtas] = ctas;
@@ -150,42 +152,117 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t *__res
     }
 }
 
-// Stand-alone split merge: one CTA of 128 threads per (column, sequence), 4 latent rows
-// per thread.  Also writes O = 0, LSE = -inf for sequences without rows.
-__global__ void __launch_bounds__(128) combine_kernel(const int32_t *__restrict__ ws, const float *__restrict__ opart,
+// Stand-alone split merge: one CTA of 128 threads per (column, sequence), 4 latent rows per
+// thread.  Up to 8 splits' partial LSEs and outputs are loaded at once, so that a sequence with
+// at most 8 splits costs one round trip to L2 once its partials are complete.  Also writes
+// O = 0, LSE = -inf for sequences without rows.
+//   spin = 0: launched after the decode (or by the caller after MLA_FLAG_SKIP_COMBINE): waits
+//             for the whole previous grid (griddepcontrol.wait) and reads the schedule the
+//             decode recorded.
+//   spin = 1: a programmatic dependent of the duo decode kernel that starts on the SMs its CTAs
+//             leave: each CTA waits only for the split counters of its own sequence and column
+//             group (both CTAs of every split add 1 with release semantics once their partials
+//             are stored), so early sequences merge while the decode still runs.
+// Either way, for the duo schedule the last combine CTA of a sequence rearms its counters.
+constexpr int kCombineBatch = 8;
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__global__ void __launch_bounds__(128) combine_kernel(int32_t *__restrict__ ws, const float *__restrict__ opart,
                                                       const float *__restrict__ lsepart, int ncols, WsLayout lay,
-                                                      __nv_bfloat16 *__restrict__ o, float *__restrict__ lse) {
+                                                      __nv_bfloat16 *__restrict__ o, float *__restrict__ lse, int spin,
+                                                      unsigned long long wait_limit_ns) {
+    if (!spin) asm volatile("griddepcontrol.wait;" ::: "memory");
     const int n = blockIdx.x, b = blockIdx.y;
-    // the schedule of the decode that wrote the partials
-    const int32_t *seq_info = ws + (ws[kHdrSchedUsed] == 1 ? lay.duo.seq_info : lay.pair.seq_info) / 4;
-    const int nsplit = seq_info[4 * b + 2];
+    // the schedule of the decode that wrote the partials (the plan's tables: complete before the
+    // decode started)
+    const bool duo = spin || __ldcg(ws + kHdrSchedUsed) == 1;
+    const Sched &sc = duo ? lay.duo : lay.pair;
+    const int32_t *seq_info = ws + sc.seq_info / 4;
+    const int nsplit = __ldcg(seq_info + 4 * b + 2);
     if (nsplit == 1) return;  // written by the decode kernel
+    int32_t *cnt = nullptr;
+    if (duo && nsplit >= 2) {
+        const int gcols = __ldcg(ws + kHdrDuo + kSchGroupCols), groups = __ldcg(ws + kHdrDuo + kSchGroups);
+        cnt = ws + sc.counters / 4 + ((int64_t)b * groups + n / gcols) * 2;
+    }
+    if (spin && nsplit >= 2) {
+        __shared__ int ready;
+        if (threadIdx.x == 0) {
+            const uint64_t t0 = global_timer_ns();
+            int ok = 1;
+            while (ld_acquire_gpu(cnt) < nsplit || ld_acquire_gpu(cnt + 1) < nsplit) {
+                if (global_timer_ns() - t0 > wait_limit_ns) {
+                    atomicCAS(ws + kHdrStatus, 0, kStatusTimeout);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(256);
+            }
+            ready = ok;
+        }
+        __syncthreads();  // with thread 0's acquire, orders every thread's reads of the partials
+        if (!ready) return;
+    }
     const int64_t orow = ((int64_t)b * ncols + n) * kDv + 4 * threadIdx.x;
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     float lse_tot = -INFINITY;
     if (nsplit >= 2) {
         const int s0 = seq_info[4 * b + 3];
         const float *l = lsepart + (int64_t)s0 * ncols + n;
-        lse_tot = merged_lse([&](int s) { return __ldcg(l + (int64_t)s * ncols); }, nsplit);
+        const float *op = opart + ((int64_t)s0 * ncols + n) * kDv + 4 * threadIdx.x;
+        float ls[kCombineBatch];
+        float4 v[kCombineBatch];
+#pragma unroll
+        for (int u = 0; u < kCombineBatch; ++u) {
+            const int su = u < nsplit ? u : nsplit - 1;
+            ls[u] = __ldcg(l + (int64_t)su * ncols);
+            v[u] = __ldcg(reinterpret_cast<const float4 *>(op + (int64_t)su * ncols * kDv));
+        }
+        if (nsplit <= kCombineBatch) {
+            lse_tot = merged_lse([&](int s) { return ls[s]; }, nsplit);
+        } else {
+            lse_tot = merged_lse([&](int s) { return __ldcg(l + (int64_t)s * ncols); }, nsplit);
+        }
+        // the sum runs in split order, as in the decode kernel's own merge
         if (lse_tot != -INFINITY) {
-            for (int s = 0; s < nsplit; ++s) {
+#pragma unroll
+            for (int u = 0; u < kCombineBatch; ++u) {
+                if (u < nsplit) {
+                    const float w = merge_weight(ls[u], lse_tot);
+                    acc[0] = fmaf(w, v[u].x, acc[0]);
+                    acc[1] = fmaf(w, v[u].y, acc[1]);
+                    acc[2] = fmaf(w, v[u].z, acc[2]);
+                    acc[3] = fmaf(w, v[u].w, acc[3]);
+                }
+            }
+            for (int s = kCombineBatch; s < nsplit; ++s) {
                 const float w = merge_weight(__ldcg(l + (int64_t)s * ncols), lse_tot);
-                const float4 v = __ldcg(reinterpret_cast<const float4 *>(opart + ((int64_t)(s0 + s) * ncols + n) * kDv +
-                                                                          4 * threadIdx.x));
-                acc[0] = fmaf(w, v.x, acc[0]);
-                acc[1] = fmaf(w, v.y, acc[1]);
-                acc[2] = fmaf(w, v.z, acc[2]);
-                acc[3] = fmaf(w, v.w, acc[3]);
+                const float4 vs = __ldcg(reinterpret_cast<const float4 *>(op + (int64_t)s * ncols * kDv));
+                acc[0] = fmaf(w, vs.x, acc[0]);
+                acc[1] = fmaf(w, vs.y, acc[1]);
+                acc[2] = fmaf(w, vs.z, acc[2]);
+                acc[3] = fmaf(w, vs.w, acc[3]);
             }
         }
     }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
     uint2 packed;
-    packed.x = *reinterpret_cast<uint32_t *>(&lo);
-    packed.y = *reinterpret_cast<uint32_t *>(&hi);
+    packed.x = *reinterpret_cast<const uint32_t *>(&lo);
+    packed.y = *reinterpret_cast<const uint32_t *>(&hi);
     *reinterpret_cast<uint2 *>(o + orow) = packed;
-    if (threadIdx.x == 0) lse[(int64_t)b * ncols + n] = lse_tot;
+    if (threadIdx.x == 0) {
+        lse[(int64_t)b * ncols + n] = lse_tot;
+        if (cnt && atomicAdd(ws + sc.done / 4 + b, 1) == ncols - 1) {
+            // every combine CTA of this sequence is past its wait: rearm for the next decode
+            const int groups = __ldcg(ws + kHdrDuo + kSchGroups);
+            for (int i = 0; i < 2 * groups; ++i) ws[sc.counters / 4 + (int64_t)b * groups * 2 + i] = 0;
+            ws[sc.done / 4 + b] = 0;
+        }
+    }
 }
 
 }  // namespace mla

@@ -90,7 +90,8 @@ struct Sched {
     size_t cta_seq;     // int32 [ctas]: the sequence that holds the unit's first tile (batch if none)
     size_t tile_off;    // int32 [batch + 1]: first flattened unit of each sequence
     size_t seq_info;    // int32 [batch][4]: units, first CTA, splits, slot offset
-    size_t counters;    // int32 [batch][groups][2 ranks]: split CTAs done, for the in-kernel merge
+    size_t counters;    // int32 [batch][groups][2 ranks]: split CTAs done (in-kernel merge, or the combine's wait)
+    size_t done;        // int32 [batch]: combine CTAs done with a sequence (the last one rearms its counters)
     int ctas_max, groups_max, unit_rows;
 };
 
@@ -119,6 +120,8 @@ MLA_HD size_t sched_tables(Sched &s, size_t off, int batch, int ctas_max, int gr
     off += align256(sizeof(int32_t) * 4 * (size_t)batch);
     s.counters = off;
     off += align256(sizeof(int32_t) * 2 * (size_t)batch * groups_max);
+    s.done = off;
+    off += align256(sizeof(int32_t) * (size_t)batch);
     return off;
 }
 

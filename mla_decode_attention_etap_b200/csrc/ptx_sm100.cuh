@@ -123,12 +123,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t remote_bar
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
-// Cluster barrier whose arrive carries no ordering of its own: the caller orders what must be
-// visible before it (a fence by one thread after a CTA barrier, which is cumulative).
+// Cluster barrier whose arrive carries no ordering of its own: for callers that have already
+// observed everything the barrier would have to order.
 __device__ __forceinline__ void cluster_sync_relaxed_arrive() {
     asm volatile("barrier.cluster.arrive.relaxed;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
-__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+// Atomic add with release semantics at GPU scope (no value returned).
+__device__ __forceinline__ void red_add_release_gpu(int32_t *p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {

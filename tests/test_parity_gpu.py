@@ -210,9 +210,11 @@ def test_bounded_waits_report_timeout_and_context_survives():
 
 @pytest.mark.parametrize("heads", [16, 128])
 def test_in_kernel_merge_matches_combine_and_resets_counters(heads):
-    """The decode kernel merges split-KV partials itself (the last split CTA of a sequence does
-    it): bitwise equal to decode-with-partials + the separate combine kernel, including empty
-    sequences, and repeatable without a new plan (the merge counters reset themselves)."""
+    """The fused call merges split-KV partials itself (h = 16: the last split CTA of a sequence in
+    the decode kernel; h = 128: the combine kernel started on the SMs the decode leaves, waiting on
+    per-sequence split counters): bitwise equal to decode-with-partials + the separate combine
+    kernel, including empty sequences, and repeatable without a new plan, before and after a
+    call that skipped the merge (the counters rearm themselves)."""
     from mla_decode_attention_etap_b200 import FLAG_SKIP_COMBINE, mla_combine
     lens = [0, 5000, 1, 2900, 0, 777]
     w = W.make_workload(len(lens), heads, lens, seed=17, paged=heads == 128)
@@ -235,7 +237,13 @@ def test_in_kernel_merge_matches_combine_and_resets_counters(heads):
     l_s = torch.full(shape, float("nan"), dtype=torch.float32, device=dev)
     dec.fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o=o_s, lse=l_s, flags=FLAG_SKIP_COMBINE)
     mla_combine(dec.workspace, w.batch, w.q_len, w.num_heads, dec.n_sms, o_s, l_s)
+    for _ in range(2):  # fused calls again after the split path
+        o = torch.full(shape + (512,), float("nan"), dtype=torch.bfloat16, device=dev)
+        lse = torch.full(shape, float("nan"), dtype=torch.float32, device=dev)
+        dec.fwd(q, kv, sl, bt, w.softmax_scale, w.causal, o=o, lse=lse)
+        outs.append((o.float().cpu().numpy(), lse.cpu().numpy()))
     torch.cuda.synchronize()
+    assert dec.status() == 0
     for o, l in outs:
         np.testing.assert_array_equal(o, o_s.float().cpu().numpy())
         np.testing.assert_array_equal(l, l_s.cpu().numpy())
@@ -258,6 +266,8 @@ def _sched_offsets(off, batch, ctas_max, groups_max):
     off += _a256(4 * 4 * batch)
     t["counters"] = off
     off += _a256(4 * 2 * batch * groups_max)
+    t["done"] = off
+    off += _a256(4 * batch)
     return t, off
 
 
