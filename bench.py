@@ -48,13 +48,24 @@ L2_BYTES = 126e6              # B200 L2: workloads below this are timed with an 
 FLUSH_BYTES = 256 << 20       # the flush writes a buffer twice the L2 size
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-KERNEL_SOURCES = ["mla_decode_attention_etap_b200/csrc/etap_pair_kernel.cuh",
-                  "mla_decode_attention_etap_b200/csrc/etap_common.cuh",
-                  "mla_decode_attention_etap_b200/csrc/ptx_sm100.cuh",
-                  "mla_decode_attention_etap_b200/csrc/plan_core.h",
-                  "mla_decode_attention_etap_b200/csrc/merge.cuh"]
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "etap_pair_kernel_ncu.md")
-PROFILE_SUMMARIES = [PROFILE_SUMMARY, os.path.join(ROOT, "profiles", "etap_pair_kernel_e4m3_ncu.md")]
+_CSRC = "mla_decode_attention_etap_b200/csrc/"
+# The sources each decode kernel is built from (its ncu traffic figure is valid while they hash the same).
+KERNEL_SOURCES = {
+    "etap_pair_kernel": [_CSRC + f for f in ("etap_pair_kernel.cuh", "etap_common.cuh", "ptx_sm100.cuh",
+                                             "plan_core.h", "merge.cuh")],
+    "etap_duo_kernel": [_CSRC + f for f in ("etap_duo_kernel.cuh", "etap_common.cuh", "ptx_sm100.cuh",
+                                            "plan_core.h", "plan_combine_kernels.cuh", "merge.cuh")],
+}
+PROFILE_SUMMARIES = {
+    "etap_pair_kernel": [os.path.join(ROOT, "profiles", "etap_pair_kernel_ncu.md"),
+                         os.path.join(ROOT, "profiles", "etap_pair_kernel_e4m3_ncu.md")],
+    "etap_duo_kernel": [os.path.join(ROOT, "profiles", "etap_duo_kernel_ncu.md")],
+}
+
+
+def decode_kernel_of(ncols: int, fp8: bool) -> str:
+    """The decode kernel a shape runs on (plan_core.h: uses_duo)."""
+    return "etap_duo_kernel" if (not fp8 and ncols > 16) else "etap_pair_kernel"
 
 WORKLOADS = {
     "b16_h16_64k": dict(batch=16, heads=16, seqlen=65536),
@@ -169,10 +180,10 @@ def code_only(text: str) -> str:
     return "\n".join(out)
 
 
-def kernel_source_hash(read=None) -> str:
-    """Hash of the decode kernel's sources (code only, so that comment edits keep a profile valid)."""
+def kernel_source_hash(read=None, kernel: str = "etap_pair_kernel") -> str:
+    """Hash of a decode kernel's sources (code only, so that comment edits keep a profile valid)."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         if read is None:
             with open(os.path.join(ROOT, rel)) as f:
                 text = f.read()
@@ -182,15 +193,15 @@ def kernel_source_hash(read=None) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, kernel: str = "etap_pair_kernel"):
     """DRAM bytes per decode launch from the committed ncu summaries, if taken on the current kernel source."""
-    for path in PROFILE_SUMMARIES:
+    for path in PROFILE_SUMMARIES[kernel]:
         try:
             text = open(path).read()
         except OSError:
             continue
         src = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
-        if not src or src.group(1) != kernel_source_hash():
+        if not src or src.group(1) != kernel_source_hash(kernel=kernel):
             continue
         m = re.search(rf"traffic_bytes_per_launch\[{re.escape(workload)}\]:\s*([0-9.eE+]+)", text)
         if m:
@@ -396,7 +407,8 @@ def run_ours(args):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
 
     def decode(q_, kv_, sl_, bt_, ql_, sc_=None):
-        # the decode kernel merges the split-KV partials itself (no combine launch)
+        # the fused call: the split-KV merge runs inside the pair kernel, or in the combine kernel that
+        # the M = 256 path launches behind its decode
         if fp8:
             mla.mla_decode_fwd_fp8(q_, kv_, sc_, sl_, bt_, w.softmax_scale, w.causal, o, lse, dec.workspace,
                                    dec.n_sms, 0, q_lens=ql_)
@@ -550,7 +562,9 @@ def run_ours(args):
         kern_s = kb0.elapsed_time(kb1) / 1e3 / n_kern
     step_s_max = reduce_max(step_s, dev)
     kern_all = [a.elapsed_time(b) / 1e3 for a, b in ev[:n_kern]]
-    launches = 2 * args.steps  # plan + decode (with the in-kernel split merge) per step
+    # plan + decode per step, + the combine kernel behind the M = 256 decode (the pair kernel merges
+    # its splits itself at n_sms = 148)
+    launches = (3 if decode_kernel_of(q_len * h, fp8) == "etap_duo_kernel" else 2) * args.steps
 
     # ---------------- end to end through the C ABI: pinned host inputs in, outputs back, every step
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -610,7 +624,8 @@ def run_ours(args):
         else:
             ach = flops / kern_s / 1e12
             roof = {"bound": "tensor", "achieved": ach, "peak": tc_tflops, "unit": "TFLOP/s", "frac": ach / tc_tflops}
-        roof["traffic"] = profiled_traffic(wname)
+        kname = decode_kernel_of(q_len * h, fp8)
+        roof["traffic"] = profiled_traffic(wname, kname)
         roof["peak_source"] = (f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
                                + ("; tensor peak = 2 x the measured bf16 GEMM peak (E4M3 operands, the nominal "
                                   "fp8 : bf16 ratio)" if fp8 else ""))
@@ -622,7 +637,11 @@ def run_ours(args):
         else:
             roof["attainable_read_gbs"] = None
             roof["attainable_note"] = "no streaming probe for the E4M3 cache's read pattern"
-        roof["kernel"] = "etap_pair_kernel<PairCfg16E4>" if fp8 else "etap_pair_kernel"
+        if kname == "etap_duo_kernel":
+            roof["kernel"] = ("etap_duo_kernel + combine_kernel (the split merge, started on the SMs the decode "
+                              "leaves; both inside the events)")
+        else:
+            roof["kernel"] = "etap_pair_kernel<PairCfg16E4>" if fp8 else "etap_pair_kernel"
         roof["kernel_ms"] = kern_s * 1e3
         roof["kernel_ms_isolated_mean"] = statistics.mean(kern_all) * 1e3
         roof["kernel_ms_isolated_median"] = statistics.median(kern_all) * 1e3
