@@ -195,7 +195,7 @@ def kernel_source_hash(read=None, kernel: str = "etap_pair_kernel") -> str:
 
 def profiled_traffic(workload: str, kernel: str = "etap_pair_kernel"):
     """DRAM bytes per decode launch from the committed ncu summaries, if taken on the current kernel source."""
-    for path in PROFILE_SUMMARIES[kernel]:
+    for path in PROFILE_SUMMARIES.get(kernel, []):
         try:
             text = open(path).read()
         except OSError:
@@ -389,6 +389,8 @@ def run_ours(args):
     mla.lib()  # fails loudly when the CUDA library is missing
 
     w, wname = make_workload(args.workload, rank, dev)
+    if args.form == "untransposed" and (w.fp8 or w.q_lens is not None):
+        raise SystemExit("--form untransposed: bf16 cache with one q_len for every sequence only")
     q, kv, sl = w.q, w.kv, w.seqlens.to(dev)
     bt = w.block_table.to(dev) if w.block_table is not None else None
     B, q_len, h = w.batch, w.q_len, w.num_heads
@@ -409,7 +411,10 @@ def run_ours(args):
     def decode(q_, kv_, sl_, bt_, ql_, sc_=None):
         # the fused call: the split-KV merge runs inside the pair kernel, or in the combine kernel that
         # the M = 256 path launches behind its decode
-        if fp8:
+        if args.form == "untransposed":
+            mla.mla_decode_fwd_untransposed(q_, kv_, sl_, bt_, w.softmax_scale, w.causal, o, lse, dec.workspace,
+                                            dec.n_sms, 0)
+        elif fp8:
             mla.mla_decode_fwd_fp8(q_, kv_, sc_, sl_, bt_, w.softmax_scale, w.causal, o, lse, dec.workspace,
                                    dec.n_sms, 0, q_lens=ql_)
         else:
@@ -417,7 +422,10 @@ def run_ours(args):
                                q_lens=ql_)
 
     def decode_on(strm):
-        if fp8:
+        if args.form == "untransposed":
+            mla.mla_decode_fwd_untransposed(q, kv, sl, bt, w.softmax_scale, w.causal, o, lse, dec.workspace,
+                                            dec.n_sms, 0, strm)
+        elif fp8:
             mla.mla_decode_fwd_fp8(q, kv, kv_scale, sl, bt, w.softmax_scale, w.causal, o, lse, dec.workspace,
                                    dec.n_sms, 0, strm, q_lens=q_lens)
         else:
@@ -564,7 +572,8 @@ def run_ours(args):
     kern_all = [a.elapsed_time(b) / 1e3 for a, b in ev[:n_kern]]
     # plan + decode per step, + the combine kernel behind the M = 256 decode (the pair kernel merges
     # its splits itself at n_sms = 148)
-    launches = (3 if decode_kernel_of(q_len * h, fp8) == "etap_duo_kernel" else 2) * args.steps
+    launches = (3 if (decode_kernel_of(q_len * h, fp8) == "etap_duo_kernel" or args.form == "untransposed")
+                else 2) * args.steps
 
     # ---------------- end to end through the C ABI: pinned host inputs in, outputs back, every step
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -624,7 +633,7 @@ def run_ours(args):
         else:
             ach = flops / kern_s / 1e12
             roof = {"bound": "tensor", "achieved": ach, "peak": tc_tflops, "unit": "TFLOP/s", "frac": ach / tc_tflops}
-        kname = decode_kernel_of(q_len * h, fp8)
+        kname = "untransposed_kernel" if args.form == "untransposed" else decode_kernel_of(q_len * h, fp8)
         roof["traffic"] = profiled_traffic(wname, kname)
         roof["peak_source"] = (f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
                                + ("; tensor peak = 2 x the measured bf16 GEMM peak (E4M3 operands, the nominal "
@@ -637,7 +646,10 @@ def run_ours(args):
         else:
             roof["attainable_read_gbs"] = None
             roof["attainable_note"] = "no streaming probe for the E4M3 cache's read pattern"
-        if kname == "etap_duo_kernel":
+        if kname == "untransposed_kernel":
+            roof["kernel"] = ("untransposed_kernel + combine_kernel (S = Q K^T form for the A/B comparison; both "
+                              "inside the events)")
+        elif kname == "etap_duo_kernel":
             roof["kernel"] = ("etap_duo_kernel + combine_kernel (the split merge, started on the SMs the decode "
                               "leaves; both inside the events)")
         else:
@@ -672,6 +684,7 @@ def run_ours(args):
             "scaling": "weak",
             "vs_baseline": None,
             "dtype": "e4m3" if fp8 else "bf16",
+            "form": args.form,
             "data": "synthetic",
             "tflops": weak_scaling_value(flops, world, step_s_max) / 1e12,
             "config": {"workload": wname, "batch_per_gpu": B, "heads": h, "q_len": q_len,
@@ -756,6 +769,8 @@ def main(argv=None):
     ap.add_argument("--no-flush", action="store_true",
                     help="do not flush L2 between timed steps of workloads smaller than L2 (L2-warm numbers)")
     ap.add_argument("--reference-rows", type=int, default=4096)
+    ap.add_argument("--form", choices=["etap", "untransposed"], default="etap",
+                    help="time the untransposed S = Q K^T decode instead of ETAP (the form comparison)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
     if args.ablation:

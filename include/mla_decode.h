@@ -178,6 +178,26 @@ MLA_API int mla_decode_fwd_fp8(const void *q, const void *kv8, const float *kv_s
                        void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream);
 
 /*
+ * The same decode in the untransposed form the pages set ETAP against ([TS]
+ * Problem Statement: S = Q K^T puts the heads on the MMA's M dimension, which the
+ * tensor core pads to its minimum; Methodology: ETAP puts the KV length there
+ * instead).  Built for the A/B comparison of the two forms on tcgen05, not for
+ * speed: M = the query-column group padded to 64 (q_len * num_heads <= 64, so
+ * 16 heads pay 4x padding) or 128, a row softmax, O = P V; two CTAs per work unit
+ * each compute all of S and one 256-column half of O (S and that half fill the
+ * TMEM).  Same plan, workspace, split-KV partials and combine as mla_decode_fwd,
+ * whose arguments, layouts, masking, outputs and errors it shares, with two
+ * limits: the bf16 cache only and one q_len for every sequence.  Any q_len *
+ * num_heads up to MLA_MAX_COLUMNS (groups of 16, 64 or 128 columns as the plan
+ * picks for mla_decode_fwd).
+ */
+MLA_API int mla_decode_fwd_untransposed(const void *q, const void *kv, const int32_t *seqlens,
+                                const int32_t *block_table, int batch, int q_len, int num_heads,
+                                int64_t kv_rows, int max_blocks, float softmax_scale, int causal, void *o,
+                                float *lse, void *workspace, size_t workspace_bytes, int num_sms,
+                                unsigned flags, void *stream);
+
+/*
  * Log-sum-exp merge of the split-KV partials that mla_decode_fwd left in the
  * workspace: lse = ln sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s, for
  * every sequence split over several CTAs; also writes O = 0, LSE = -inf for

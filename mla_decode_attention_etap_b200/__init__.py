@@ -29,7 +29,7 @@ STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3:
 EXPORTS = ("mla_decode_workspace_size", "mla_decode_plan", "mla_decode_fwd", "mla_combine",
            "mla_decode_read_status", "mla_decode_plan_host", "mla_status_string", "mla_last_cuda_error",
            "mla_decode_fwd_static_ws", "mla_decode_static_ws_status", "mla_decode_fwd_ragged", "mla_stream_probe", "mla_decode_fwd_fp8", "mla_form_ablation",
-           "mla_decode_fwd_trace")
+           "mla_decode_fwd_trace", "mla_decode_fwd_untransposed")
 STATIC_WORKSPACE_BYTES = 16777216
 
 
@@ -64,6 +64,9 @@ def lib() -> ctypes.CDLL:
         L.mla_decode_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp,
                                          vp, vp, sz, i32, ctypes.c_uint, vp]
         L.mla_decode_fwd_fp8.restype = i32
+        L.mla_decode_fwd_untransposed.argtypes = [vp, vp, vp, vp, i32, i32, i32, i64, i32, ctypes.c_float, i32, vp,
+                                                  vp, vp, sz, i32, ctypes.c_uint, vp]
+        L.mla_decode_fwd_untransposed.restype = i32
         L.mla_combine.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
         L.mla_combine.restype = i32
         L.mla_decode_read_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int), vp]
@@ -199,6 +202,24 @@ def mla_decode_fwd(q, kv, seqlens, block_table, softmax_scale, causal, o, lse, w
                                            _ptr(o), _ptr(lse), _ptr(workspace),
                                            workspace.numel() * workspace.element_size(), n_sms, flags,
                                            _stream(stream)), "mla_decode_fwd_ragged")
+
+
+def mla_decode_fwd_untransposed(q, kv, seqlens, block_table, softmax_scale, causal, o, lse, workspace, n_sms,
+                                flags=0, stream=None) -> None:
+    """The same decode in the untransposed form, S = Q K^T with the query columns on M (padded to 64
+    or 128): the form the pages set ETAP against, for the A/B comparison (``mla_decode_fwd_untransposed``;
+    bf16 cache, one q_len for every sequence)."""
+    _require_cuda(q, "q")
+    check_decode_args(q, kv, seqlens, block_table, o, lse, workspace)
+    B, q_len, h, _ = q.shape
+    if block_table is not None:
+        kv_rows, max_blocks = kv.shape[0] * kv.shape[1], block_table.shape[1]
+    else:
+        kv_rows, max_blocks = kv.shape[1], 0
+    _check(lib().mla_decode_fwd_untransposed(_ptr(q), _ptr(kv), _ptr(seqlens), _ptr(block_table), B, q_len, h,
+                                             kv_rows, max_blocks, float(softmax_scale), int(bool(causal)), _ptr(o),
+                                             _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                             n_sms, flags, _stream(stream)), "mla_decode_fwd_untransposed")
 
 
 def mla_decode_fwd_fp8(q, kv8, kv_scale, seqlens, block_table, softmax_scale, causal, o, lse, workspace, n_sms,

@@ -16,6 +16,7 @@
 #include "etap_pair_kernel.cuh"
 #include "etap_duo_kernel.cuh"
 #include "plan_combine_kernels.cuh"
+#include "untransposed_kernel.cuh"
 #include "plan_core.h"
 #include "form_ablation.cuh"
 #include "stream_probe.cuh"
@@ -108,6 +109,9 @@ int ensure_smem_attr() {
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         e = cudaFuncSetAttribute(mla::etap_duo_kernel<mla::DuoCfg64, mla::DuoCfg128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::kDuoSmemAlloc);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        e = cudaFuncSetAttribute(mla::untransposed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)mla::kUtSmemAlloc);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         done[dev] = true;
     }
@@ -321,8 +325,9 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
                     const int32_t *q_lens, const int32_t *block_table, int batch, int q_len, int num_heads,
                     int64_t kv_rows, int max_blocks, float softmax_scale, int causal, void *o, float *lse,
                     void *workspace, size_t workspace_bytes, int num_sms, unsigned flags, void *stream,
-                    unsigned long long *trace = nullptr, int trace_cap = 0) {
+                    unsigned long long *trace = nullptr, int trace_cap = 0, bool untransposed = false) {
     const bool fp8 = kv_scale != nullptr;
+    if (untransposed && (fp8 || q_lens || trace)) return MLA_ERR_UNSUPPORTED;
     int st = check_shape(batch, q_len, num_heads, num_sms);
     if (st != MLA_OK) return st;
     if (!q || !kv || !seqlens || !o || !lse || !workspace) return MLA_ERR_INVALID_ARG;
@@ -414,6 +419,41 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
+    if (untransposed) {
+        // S = Q K^T form: two CTAs per work unit of the pair schedule (<= 16 columns) or the duo one
+        mla::UtMaps maps;
+        st = encode_rows_576(&maps.q64, q, (uint64_t)batch * ncols, 64);
+        if (st != MLA_OK) return st;
+        st = encode_rows_576(&maps.kv, kv, kv_total_rows, 64);
+        if (st != MLA_OK) return st;
+        p.fuse_merge = 0;
+        p.signal_combine = 0;
+        int units = lay.ctas * lay.groups;
+        if (lay.has_duo) {
+            units = 0;
+            for (int mode = 0; mode < 2; ++mode) {
+                if (mode == 1 && !mla::duo_mode1_possible(ncols)) break;
+                const int g = mla::duo_groups(ncols, mode), c = mla::num_ctas(num_sms, g) * g;
+                if (c > units) units = c;
+            }
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * units, 1, 1);
+        cfg.blockDim = dim3(mla::kUtThreads, 1, 1);
+        cfg.dynamicSmemBytes = mla::kUtSmemAlloc;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, mla::untransposed_kernel, maps, p, lay);
+        if (e != cudaSuccess) return cuda_fail(e, "untransposed_kernel launch");
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "untransposed_kernel launch");
+        if (flags & MLA_FLAG_SKIP_COMBINE) return MLA_OK;
+        return launch_combine(workspace, batch, q_len, num_heads, num_sms, o, lse, 0, p.wait_limit_ns, s);
+    }
     if (duo) {
         mla::DuoMaps maps;
         st = encode_rows_576(&maps.q32, q, (uint64_t)batch * ncols, 32);
@@ -464,6 +504,15 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
 }  // namespace
 
 extern "C" {
+
+int mla_decode_fwd_untransposed(const void *q, const void *kv, const int32_t *seqlens, const int32_t *block_table,
+                                int batch, int q_len, int num_heads, int64_t kv_rows, int max_blocks,
+                                float softmax_scale, int causal, void *o, float *lse, void *workspace,
+                                size_t workspace_bytes, int num_sms, unsigned flags, void *stream) {
+    return decode_fwd_impl(q, kv, nullptr, seqlens, nullptr, block_table, batch, q_len, num_heads, kv_rows,
+                           max_blocks, softmax_scale, causal, o, lse, workspace, workspace_bytes, num_sms, flags,
+                           stream, nullptr, 0, true);
+}
 
 int mla_decode_fwd_ragged(const void *q, const void *kv, const int32_t *seqlens, const int32_t *q_lens,
                           const int32_t *block_table, int batch, int q_len, int num_heads, int64_t kv_rows,
