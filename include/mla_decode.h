@@ -221,16 +221,17 @@ MLA_API int mla_stream_probe(const void *kv, int64_t rows, int units, int32_t *e
 
 /*
  * Measurement helper, not part of the decode (the pages have no counterpart): mla_decode_fwd
- * (flags 0) that also records when each role of the two CTAs of cluster 0 reached its events, so
- * that the pipeline of the M = 256 kernel (bf16 cache, q_len*h > 16) can be read off one launch.
+ * (flags 0, bf16 cache) that also records when each role of the two CTAs of cluster 0 reached its
+ * events, so that a kernel's pipeline can be read off one launch.
  *   trace      device uint64 [2 CTAs][5 roles][trace_cap], then [num_sms][4]: 8-byte aligned,
- *              zeroed by the caller; roles: 0 K-tile producer, 1 step-1 MMA issuer (CTA 0 only),
- *              2 value producer, 3 softmax, 4 step-3 MMA issuer (CTA 0 only).  The trailing
- *              rows hold each CTA's %globaltimer (ns) at entry, start of work (the plan read),
- *              end of work and exit.
+ *              zeroed by the caller.  Roles of the M = 256 kernel (q_len*h > 16): 0 K-tile
+ *              producer, 1 step-1 MMA issuer (CTA 0 only), 2 value producer, 3 softmax, 4 step-3
+ *              MMA issuer (CTA 0 only); of the CTA-pair kernel (q_len*h <= 16): 0 producer,
+ *              1 MMA issuer, 3 softmax.  The trailing rows hold each CTA's %globaltimer (ns) at
+ *              entry, start of work (the plan read), end of work and exit.
  *              Entry = (event code << 56) | (index << 40) | (%globaltimer ns mod 2^40); a role
  *              stops recording after trace_cap events.  The event codes are listed in
- *              etap_duo_kernel.cuh.  Other shapes run the untraced kernels and leave it as it is.
+ *              etap_duo_kernel.cuh and etap_common.cuh (the pair kernel's).
  *   trace_cap  1 .. 2^20
  * All other arguments, results and errors as for mla_decode_fwd.  The stamps cost a few
  * instructions per event in those four threads.

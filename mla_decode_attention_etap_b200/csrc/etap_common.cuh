@@ -68,6 +68,21 @@ struct DecodeParams {
 // Event stamps for the tracing entry point: (code << 56) | (index << 40) | (globaltimer ns mod 2^40),
 // written by one thread per (CTA, role) of cluster 0 into its own row of the trace buffer.
 enum : int { kTraceRoles = 5 };
+// Events of the CTA-pair kernel (softmax role, row 3): tile k's scores in / its P^T handed to
+// step 3 (index: tile), a segment's epilogue begins / its last step 3 is complete / its outputs or
+// partials are stored (index: splits) / this CTA merges the splits (index: splits) / it ends.
+enum : int {
+    kPairEvTile = 50,
+    kPairEvTileDone = 51,
+    kPairEvEpi = 52,
+    kPairEvEpiS3 = 53,
+    kPairEvEpiO = 54,
+    kPairEvMerge = 55,
+    kPairEvEpiDone = 56,
+    kPairEvQ = 57,       // producer (row 0): a segment's Q loads issued (index: segment)
+    kPairEvPair = 58,    // producer (row 0): a value pair's loads issued (index: pair)
+    kPairEvScores = 59   // MMA issuer (row 1): a tile's score MMAs issued and committed (index: tile)
+};
 struct TraceRow {
     unsigned long long *row;
     int n, cap;

@@ -977,8 +977,7 @@ __global__ void __launch_bounds__(kDuoThreads, 1)
     // No CTA leaves while its peer may still write into its shared memory.  Every operation that
     // targets a CTA's shared memory (TMA bytes, st.async, remote and multicast arrivals) has been
     // waited for by that CTA above (the producers' tails included), so the barrier needs no
-    // ordering of its own: a releasing arrive would wait for every global store of the CTA, tens
-    // of microseconds while the memory system is busy.
+    // ordering of its own.
     cluster_sync_relaxed_arrive();
     if (wc->abort) {
         // After an abort a peer's last st.async or bulk copy may not have been waited for: let it

@@ -210,6 +210,9 @@ __global__ void __launch_bounds__(320, 1)
     auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * (uint32_t)i; };
     volatile WaitCtl *wc = reinterpret_cast<volatile WaitCtl *>(smem + C::OFF_MISC + 16);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    // trace: every CTA's entry, start of work (after the plan), end of work and exit
+    unsigned long long *span = p.trace ? p.trace + (size_t)2 * kTraceRoles * p.trace_cap + 4 * (size_t)blockIdx.x : nullptr;
+    if (span && threadIdx.x == 0) span[0] = global_timer_ns();
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::NV; ++i) {
@@ -307,6 +310,7 @@ __global__ void __launch_bounds__(320, 1)
     // A programmatic dependent launched next (the next plan) may be scheduled from now on; it
     // waits for this grid to complete before touching memory.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (span && threadIdx.x == 0) span[1] = global_timer_ns();
 
     // The schedule must come from a plan for this same grid (uniform in the whole cluster).
     const bool plan_ok = p.ws[kHdrPair + kSchCtas] == p.ctas && p.ws[kHdrPair + kSchGroups] == p.groups &&
@@ -338,6 +342,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < C::NR; ++i) arms_r[i] = 0;
         int arms_q = 0, tail_uses = 0;
         bool ok = true;
+        TraceRow trp;  // cluster 0: Q and value-pair loads issued
+        trp.init(p, 0);
+        if (lane != 0) trp.row = nullptr;
         // L2 prefetch of this CTA's columns of a future tile, so that the load that
         // refills a freed slot hits L2 instead of waiting on HBM.
         auto prefetch_tile = [&](int pb_, int pt_) {
@@ -388,6 +395,7 @@ __global__ void __launch_bounds__(320, 1)
                                     qrow);
                     tma_load_2d(sbase + C::OFF_QR, &tm_qr, bar(BR::QFULL), rope_x, qrow);
                 }
+                trp.put(kPairEvQ, seg);
                 if (!C::KV8 && !p.withhold_q) ++arms_q;
                 for (int t = t0 + toff; t < t1 && ok; t += C::TSTEP, ++k) {
                     if (lane == 0 && ahead.valid) {
@@ -459,6 +467,7 @@ __global__ void __launch_bounds__(320, 1)
                                         tma_load_2d(dst + hc * C::CHUNK + hh * C::HALF, &tm_kv, bar(BR::VFULL + vs),
                                                     x0 + C::CHUNK_COLS * hc, y[hh]);
                             }
+                            trp.put(kPairEvPair, g2);
                             ++phases_v[vs];
                             tma_v[vs] = true;
                         } else {
@@ -513,6 +522,8 @@ __global__ void __launch_bounds__(320, 1)
         // after the scores' MMAs, so the softmax of tile k overlaps step 3 of
         // tile k-1 on the tensor pipe.
         if (lane == 0 && fb < fe) {
+            TraceRow tri;  // cluster 0: score MMAs of a tile issued and committed
+            tri.init(p, 1);
             const uint32_t q_base = sbase + C::OFF_Q;
             // one 128-byte chunk of K-major operands: four 32-byte K-steps (16 bf16 or 32 E4M3)
             auto qk_chunk = [&](uint32_t d_s, uint32_t a_base, int qchunk, bool init) {
@@ -584,6 +595,7 @@ __global__ void __launch_bounds__(320, 1)
                             progressed = true;
                             if (++qstage > C::PAIRS) {
                                 umma_commit(bar(BR::SFULL + (kq & 1)));
+                                tri.put(kPairEvScores, kq);
                                 if (qc.last()) {
                                     umma_commit(bar(BR::QEMPTY));
                                     ++seg_q;
@@ -629,6 +641,9 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t xfree_remote = map_to_rank(bar(BR::XFREE + sw), peer);
         const int k_total = (int)(fe - fb);
         bool ok = true, stop = false, pv_issued = false;
+        TraceRow tr;  // cluster 0: one softmax thread stamps the tile and epilogue events
+        tr.init(p, 3);
+        if (warp != 2 || lane != 0) tr.row = nullptr;
         // Exchange slots hold 128 rows x 16 fp32; this thread's 8 values are 16-byte chunks 2*half, 2*half+1.
         auto x_off = [&](int j) -> uint32_t { return swz_off(row, 2 * half + j, 64, 3); };
         // CH > 1: whole-tile exchange, one tile ahead.  Our partial S^T of tile kk goes to the
@@ -784,6 +799,7 @@ __global__ void __launch_bounds__(320, 1)
                     const int pb = k % C::PB;
                     ok = ok && spin_phase<false>(bar(BR::SFULL + (k & 1)), (k >> 1) & 1, wc, status);
                     tc_fence_after();
+                    tr.put(kPairEvTile, k);
                     const int rg = t * kTileRows + row;
                     // E4M3: this row's scale s (from the rope slot, which the warps then free); the row's scores
                     // are s * (K codes . Q terms) * 2^-c_n, and the maximum tracks them plus log2 s
@@ -1079,6 +1095,7 @@ __global__ void __launch_bounds__(320, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(BR::PFULL + pb));
                     }
+                    tr.put(kPairEvTileDone, k);
                     if constexpr (C::CH > 1 && !C::KV8) {
                         if (k + 1 < k_total && !sent_next) send_tile(k + 1);
                     }
@@ -1086,9 +1103,11 @@ __global__ void __launch_bounds__(320, 1)
                 if (stop) break;
                 // ---------------------------------------------------- epilogue: step 4 for this CTA's 256 columns
                 const int kl = k - 1;
+                tr.put(kPairEvEpi, seg);
                 if (has_tiles)  // the last step 3 of this segment has completed
                     ok = ok && spin_phase<false>(bar(BR::PEMPTY + (kl % C::PB)), (kl / C::PB) & 1, wc, status);
                 tc_fence_after();
+                tr.put(kPairEvEpiS3, seg);
 #pragma unroll
                 for (int ch = 0; ch < C::CH; ++ch) {
                     float v8[8];
@@ -1248,6 +1267,7 @@ __global__ void __launch_bounds__(320, 1)
                     store_lse(ch, lse_n);
                 }
                 }
+                tr.put(kPairEvEpiO, nsplit);
                 if (nsplit >= 2 && p.fuse_merge) {
                     // Split-KV merge in the kernel: the last CTA (of this rank) to finish a split of
                     // sequence b merges all splits for its 256 latent rows and this column group.
@@ -1264,6 +1284,7 @@ __global__ void __launch_bounds__(320, 1)
                     }
                     named_bar_sync(SMX, NSM);
                     if (*merge_flag) {
+                        tr.put(kPairEvMerge, nsplit);
                         // thread = 4 consecutive latent rows (one float4) x NG/4 columns.  The first
                         // U splits' partial outputs are in flight while the LSE partials are staged in
                         // an idle buffer (bf16: the P^T buffers, whose last step 3 has completed; E4M3:
@@ -1332,9 +1353,11 @@ __global__ void __launch_bounds__(320, 1)
                     }
                 }
                 tc_fence_before();
+                tr.put(kPairEvEpiDone, seg);
                 ++seg;
             }
         }
+        if (span && warp == 2 && lane == 0) span[2] = global_timer_ns();
         if (p.fuse_merge && !stop && ok) {
             // Sequences without a single KV row get no split: O = 0 and LSE = -inf, written by
             // cluster b mod (number of clusters), each CTA for its 256 latent rows.
@@ -1369,6 +1392,7 @@ __global__ void __launch_bounds__(320, 1)
     cluster_sync();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+    if (span && threadIdx.x == 32) span[3] = global_timer_ns();
 }
 
 }  // namespace mla
