@@ -233,8 +233,9 @@ MLA_API int mla_stream_probe(const void *kv, int64_t rows, int units, int32_t *e
  *              stops recording after trace_cap events.  The event codes are listed in
  *              etap_duo_kernel.cuh and etap_common.cuh (the pair kernel's).
  *   trace_cap  1 .. 2^20
- * All other arguments, results and errors as for mla_decode_fwd.  The stamps cost a few
- * instructions per event in those four threads.
+ * All other arguments, results and errors as for mla_decode_fwd.  The traced kernels are
+ * separate instances of the decode kernels; the ones the other entry points launch carry no
+ * stamps at all.
  */
 MLA_API int mla_decode_fwd_trace(const void *q, const void *kv, const int32_t *seqlens, const int32_t *block_table,
                                  int batch, int q_len, int num_heads, int64_t kv_rows, int max_blocks,

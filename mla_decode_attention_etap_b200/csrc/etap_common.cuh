@@ -83,21 +83,36 @@ enum : int {
     kPairEvPair = 58,    // producer (row 0): a value pair's loads issued (index: pair)
     kPairEvScores = 59   // MMA issuer (row 1): a tile's score MMAs issued and committed (index: tile)
 };
-struct TraceRow {
+// ON = false (the kernels the decode entry points launch) compiles every stamp away; the traced
+// instances are separate kernels, launched only by the tracing entry point.
+template <bool ON>
+struct TraceRowT {
     unsigned long long *row;
     int n, cap;
     __device__ void init(const DecodeParams &p, int role) {
         n = 0;
         cap = p.trace_cap;
-        row = (p.trace && blockIdx.x < 2) ? p.trace + ((size_t)blockIdx.x * kTraceRoles + role) * (size_t)cap : nullptr;
+        row = (ON && p.trace && blockIdx.x < 2) ? p.trace + ((size_t)blockIdx.x * kTraceRoles + role) * (size_t)cap
+                                                : nullptr;
     }
     __device__ __forceinline__ void put(int code, int index) {
-        if (row && n < cap) {
-            row[n++] = ((unsigned long long)code << 56) | ((unsigned long long)(index & 0xFFFF) << 40) |
-                       (global_timer_ns() & 0xFFFFFFFFFFull);
+        if constexpr (ON) {
+            if (row && n < cap) {
+                row[n++] = ((unsigned long long)code << 56) | ((unsigned long long)(index & 0xFFFF) << 40) |
+                           (global_timer_ns() & 0xFFFFFFFFFFull);
+            }
         }
     }
 };
+// Per-CTA stamps (entry, start of work, end of work, exit) after the role rows; nullptr unless traced.
+template <bool ON>
+__device__ __forceinline__ unsigned long long *trace_span(const DecodeParams &p) {
+    if constexpr (ON) {
+        return p.trace ? p.trace + (size_t)2 * kTraceRoles * p.trace_cap + 4 * (size_t)blockIdx.x : nullptr;
+    } else {
+        return nullptr;
+    }
+}
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA abort
 // flag) when the wait ran past kWaitLimitNs, or when another role aborted.

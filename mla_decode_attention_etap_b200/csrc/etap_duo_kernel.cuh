@@ -131,7 +131,7 @@ enum : int {
     kEvEpiO = 40        // epilogue: outputs (or partials) stored
 };
 
-template <class C>
+template <class C, bool TR>
 __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &p, uint8_t *smem, uint32_t sbase,
                                          uint32_t tmem, uint32_t rank, int unit, int grp, int groups, bool has_work,
                                          volatile WaitCtl *wc, int32_t *status, bool &pv_pending) {
@@ -207,7 +207,7 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
         // ------------------------------------------------------------ K tiles and Q (step-1 operands)
         if (lane == 0 && fb < fe) {
             bool ok = true;
-            TraceRow tr;
+            TraceRowT<TR> tr;
             tr.init(p, 0);
             SegIter it;
             it.init_at(seq0, fb, fe);
@@ -257,7 +257,7 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
         // 256 rank + 128 j .. + 127 of those rows, as one 32 KB slot of two 64-column chunks.
         if (fb < fe) {
             bool ok = true;
-            TraceRow tr;
+            TraceRowT<TR> tr;
             tr.init(p, 2);
             SegIter it;
             it.init_at(seq0, fb, fe);
@@ -337,7 +337,7 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
             qc.init(tile_off, seq0, fb, fe);
             int kq = 0, seg_q = 0, qstage = 0;
             uint32_t g1 = 0;
-            TraceRow tr;
+            TraceRowT<TR> tr;
             tr.init(p, 1);
             uint64_t t_last = global_timer_ns();
             while (qc.valid) {
@@ -414,7 +414,7 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
                 int kp = 0, pstage = 0;
                 bool armed = false;
                 uint32_t g3 = 0;
-                TraceRow tr;
+                TraceRowT<TR> tr;
                 tr.init(p, 4);
                 uint64_t t_last = global_timer_ns();
                 while (pc.valid) {
@@ -550,7 +550,7 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
         const uint32_t lx_remote = map_to_rank(sbase + kDuoCtlLx, peer);
         bool ok = true, stop = false;
         int k = 0, xmr = 0, xlr = 0;
-        TraceRow tr;
+        TraceRowT<TR> tr;
         tr.init(p, 3);
         if (tid != 0) tr.row = nullptr;
         // Scores of 32 columns of this thread's row (block cc of its half), scaled to log2 units
@@ -879,7 +879,7 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
     }
 }
 
-template <class C64, class C128>
+template <class C64, class C128, bool TR = false>
 __global__ void __launch_bounds__(kDuoThreads, 1)
     etap_duo_kernel(const __grid_constant__ DuoMaps tm, const __grid_constant__ DecodeParams p) {
     using BR = DuoBars;
@@ -895,7 +895,7 @@ __global__ void __launch_bounds__(kDuoThreads, 1)
     volatile WaitCtl *wc = reinterpret_cast<volatile WaitCtl *>(smem + kDuoCtlMisc + 16);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kDuoCtlMisc);
     // trace: every CTA's entry, start of work (after the plan), end of work and exit
-    unsigned long long *span = p.trace ? p.trace + (size_t)2 * kTraceRoles * p.trace_cap + 4 * (size_t)blockIdx.x : nullptr;
+    unsigned long long *span = trace_span<TR>(p);
     if (span && threadIdx.x == 0) span[0] = global_timer_ns();
 
     if (threadIdx.x == 0) {
@@ -961,9 +961,9 @@ __global__ void __launch_bounds__(kDuoThreads, 1)
     bool pv_pending = false;
     if (span && threadIdx.x == 0) span[1] = global_timer_ns();
     if (mode == 1)
-        duo_body<C128>(tm, p, smem, sbase, tmem, rank, unit, grp, groups, has_work, wc, status, pv_pending);
+        duo_body<C128, TR>(tm, p, smem, sbase, tmem, rank, unit, grp, groups, has_work, wc, status, pv_pending);
     else
-        duo_body<C64>(tm, p, smem, sbase, tmem, rank, unit, grp, groups, has_work, wc, status, pv_pending);
+        duo_body<C64, TR>(tm, p, smem, sbase, tmem, rank, unit, grp, groups, has_work, wc, status, pv_pending);
     if (pv_pending) {
         // every MMA issued completes before TMEM is released (one barrier per issuing thread)
         const int fin = warp == 1 ? BR::FINAL : BR::FINAL3;

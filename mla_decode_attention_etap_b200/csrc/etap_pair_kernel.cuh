@@ -186,7 +186,7 @@ __device__ __forceinline__ uint32_t swz_off(uint32_t r, uint32_t j, uint32_t pit
     return off + ((j ^ ((off >> 7) & mask)) << 4);
 }
 
-template <class C>
+template <class C, bool TR = false>
 __global__ void __launch_bounds__(320, 1)
     etap_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                      const __grid_constant__ CUtensorMap tm_qr, const __grid_constant__ CUtensorMap tm_kvr,
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(320, 1)
     volatile WaitCtl *wc = reinterpret_cast<volatile WaitCtl *>(smem + C::OFF_MISC + 16);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     // trace: every CTA's entry, start of work (after the plan), end of work and exit
-    unsigned long long *span = p.trace ? p.trace + (size_t)2 * kTraceRoles * p.trace_cap + 4 * (size_t)blockIdx.x : nullptr;
+    unsigned long long *span = trace_span<TR>(p);
     if (span && threadIdx.x == 0) span[0] = global_timer_ns();
 
     if (threadIdx.x == 0) {
@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < C::NR; ++i) arms_r[i] = 0;
         int arms_q = 0, tail_uses = 0;
         bool ok = true;
-        TraceRow trp;  // cluster 0: Q and value-pair loads issued
+        TraceRowT<TR> trp;  // cluster 0: Q and value-pair loads issued
         trp.init(p, 0);
         if (lane != 0) trp.row = nullptr;
         // L2 prefetch of this CTA's columns of a future tile, so that the load that
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(320, 1)
         // after the scores' MMAs, so the softmax of tile k overlaps step 3 of
         // tile k-1 on the tensor pipe.
         if (lane == 0 && fb < fe) {
-            TraceRow tri;  // cluster 0: score MMAs of a tile issued and committed
+            TraceRowT<TR> tri;  // cluster 0: score MMAs of a tile issued and committed
             tri.init(p, 1);
             const uint32_t q_base = sbase + C::OFF_Q;
             // one 128-byte chunk of K-major operands: four 32-byte K-steps (16 bf16 or 32 E4M3)
@@ -641,7 +641,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t xfree_remote = map_to_rank(bar(BR::XFREE + sw), peer);
         const int k_total = (int)(fe - fb);
         bool ok = true, stop = false, pv_issued = false;
-        TraceRow tr;  // cluster 0: one softmax thread stamps the tile and epilogue events
+        TraceRowT<TR> tr;  // cluster 0: one softmax thread stamps the tile and epilogue events
         tr.init(p, 3);
         if (warp != 2 || lane != 0) tr.row = nullptr;
         // Exchange slots hold 128 rows x 16 fp32; this thread's 8 values are 16-byte chunks 2*half, 2*half+1.
@@ -1229,7 +1229,9 @@ __global__ void __launch_bounds__(320, 1)
                             const float mm = fmaxf(ms[li], mp);
                             const float as = ms[li] == -INFINITY ? 0.f : fast_exp2(ms[li] - mm);
                             const float ap = mp == -INFINITY ? 0.f : fast_exp2(mp - mm);
-                            const float l = ls[li] * as + lp * ap;
+                            // rank 0's term first in both CTAs, so that both compute the same l (and LSE)
+                            const float l = rank == 0 ? __fmaf_rn(ls[li], as, __fmul_rn(lp, ap))
+                                                      : __fmaf_rn(lp, ap, __fmul_rn(ls[li], as));
                             const bool empty = !(l > 0.f) || mm == -INFINITY;
                             // the stored p carried a factor 2^4
                             const float inv = empty ? 0.f : 0.0625f / l;

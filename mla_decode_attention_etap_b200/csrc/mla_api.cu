@@ -110,6 +110,15 @@ int ensure_smem_attr() {
         e = cudaFuncSetAttribute(mla::etap_duo_kernel<mla::DuoCfg64, mla::DuoCfg128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::kDuoSmemAlloc);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        e = cudaFuncSetAttribute(mla::etap_duo_kernel<mla::DuoCfg64, mla::DuoCfg128, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::kDuoSmemAlloc);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg16, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::PairCfg16::SMEM_ALLOC);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg32, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::PairCfg32::SMEM_ALLOC);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         e = cudaFuncSetAttribute(mla::untransposed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)mla::kUtSmemAlloc);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -138,6 +147,10 @@ cudaError_t launch_pair(const CUtensorMap &tm_q, const CUtensorMap &tm_kv, const
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
+    // the traced instance only for the tracing entry point (bf16 configurations)
+    if constexpr (!C::KV8) {
+        if (p.trace) return cudaLaunchKernelEx(&cfg, mla::etap_pair_kernel<C, true>, tm_q, tm_kv, tm_qr, tm_kvr, p);
+    }
     return cudaLaunchKernelEx(&cfg, mla::etap_pair_kernel<C>, tm_q, tm_kv, tm_qr, tm_kvr, p);
 }
 
@@ -158,6 +171,7 @@ cudaError_t launch_duo(const mla::DuoMaps &maps, const mla::DecodeParams &p, int
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
+    if (p.trace) return cudaLaunchKernelEx(&cfg, mla::etap_duo_kernel<mla::DuoCfg64, mla::DuoCfg128, true>, maps, p);
     return cudaLaunchKernelEx(&cfg, mla::etap_duo_kernel<mla::DuoCfg64, mla::DuoCfg128>, maps, p);
 }
 
