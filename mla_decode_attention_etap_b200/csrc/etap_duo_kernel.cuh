@@ -666,7 +666,8 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
                         grp * NC + NC <= p.ncols;
                     // ---- pass 1: does any score exceed its column's running maximum by > 2^THRESH?
                     bool need = first || !ok;
-#pragma unroll
+                    // rolled: one copy of the score read and test (instruction cache; measured faster)
+#pragma unroll 1
                     for (int cc = 0; cc < NH / 32; ++cc) {
                         float x[32];
                         load_scores(cc, full, rg, x);
@@ -695,7 +696,7 @@ __device__ __forceinline__ void duo_body(const DuoMaps &tm, const DecodeParams &
                     if (named_bar_or(SMX, NSM, vote || peer_vote)) {
                         tr.put(kEvSmSlow, k);
                         // ---- slow path, taken by both CTAs together: tile maxima over all 256 rows
-#pragma unroll
+#pragma unroll 1
                         for (int cc = 0; cc < NH / 32; ++cc) {
                             float x[32];
                             load_scores(cc, full, rg, x);
