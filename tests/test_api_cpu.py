@@ -233,3 +233,37 @@ def test_decode_guards_accept_what_the_parity_tests_pass(kw):
         m.check_decode_args(w.q, w.kv8, w.seqlens, w.block_table, o, lse, ws, w.q_lens, kv_scale=w.kv_scale)
     else:
         m.check_decode_args(w.q, w.kv, w.seqlens, w.block_table, o, lse, ws, w.q_lens)
+
+
+def test_trace_buffer_layout_and_decoders():
+    """The trace buffer holds [2 CTAs][5 roles][cap] event words, then [n_sms][4] span stamps; the
+    decoders split them, order events by time and make spans relative to the earliest entry."""
+    cap, n_sms = 4, 3
+    t = m.trace_buffer(cap, n_sms)
+    assert t.dtype == torch.int64 and t.numel() == 2 * 5 * cap + 4 * n_sms and int(t.abs().sum()) == 0
+    rows = t[:2 * 5 * cap].view(2, 5, cap)
+    word = lambda code, idx, ns: (code << 56) | (idx << 40) | ns
+    rows[0, 3, 0] = word(50, 7, 1000)
+    rows[0, 3, 1] = word(51, 7, 1900)
+    rows[1, 0, 0] = word(57, 0, 1500)
+    spans = t[2 * 5 * cap:].view(n_sms, 4)
+    spans[0] = torch.tensor([10_000, 10_600, 30_000, 31_000])
+    spans[1] = torch.tensor([10_200, 10_700, 29_000, 29_500])
+    ev = m.decode_trace_events(t, n_sms)
+    assert [(e[0], e[1], e[2], e[3]) for e in ev] == [(0, 3, 50, 7), (1, 0, 57, 0), (0, 3, 51, 7)]
+    assert [e[4] for e in ev] == [0, 500, 900]
+    sp = m.decode_trace_spans(t, n_sms)
+    assert sp[0].tolist() == [0, 600, 20_000, 21_000] and sp[1].tolist() == [200, 700, 19_000, 19_500]
+    assert sp[2].tolist() == [0, 0, 0, 0]  # a CTA that did not run stays zero
+
+
+def test_untransposed_and_trace_entry_points_validate_on_the_host():
+    """The two measurement entry points refuse bad arguments before any launch."""
+    L = m.lib()
+    # null pointers
+    rc = L.mla_decode_fwd_untransposed(None, None, None, None, 1, 1, 16, 64, 0, ctypes.c_float(0.1), 0, None, None,
+                                       None, 0, 148, 0, None)
+    assert rc == -1
+    rc = L.mla_decode_fwd_trace(None, None, None, None, 1, 1, 16, 64, 0, ctypes.c_float(0.1), 0, None, None, None,
+                                0, 148, None, 16, None)
+    assert rc == -1

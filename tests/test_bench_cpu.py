@@ -30,3 +30,17 @@ def test_peaks_come_from_the_measured_file_else_the_recipe_fallback(monkeypatch,
     # the profiling recipe's fallback: 6.65 TB/s and 1.59 PFLOP/s (burst), about 1.4 sustained
     monkeypatch.setattr(bench, "PEAKS_FILE", str(tmp_path / "absent.json"))
     assert bench.load_peaks() == (6650.0, 1590.0, 1400.0, "fallback")
+
+
+def test_each_kernel_has_its_own_source_hash_and_summary():
+    """The traffic figure of a workload comes from the summary of the kernel that workload runs,
+    keyed on that kernel's own sources."""
+    assert bench.decode_kernel_of(16, False) == "etap_pair_kernel"
+    assert bench.decode_kernel_of(17, False) == "etap_duo_kernel"
+    assert bench.decode_kernel_of(128, True) == "etap_pair_kernel"  # the FP8 cache keeps the pair kernel
+    assert bench.kernel_source_hash(kernel="etap_pair_kernel") != bench.kernel_source_hash(kernel="etap_duo_kernel")
+    assert bench.profiled_traffic("mla_decode_b16_h16_q1_L65536_contiguous", "etap_duo_kernel") is None
+    assert bench.profiled_traffic("anything", "untransposed_kernel") is None
+    t = bench.profiled_traffic("mla_decode_b32_h128_q1_Lunif8192to32768_paged64", "etap_duo_kernel")
+    assert t is not None and 1.0 <= t / 785979648 < 1.2  # the value re-read adds up to ~10% of HBM reads
+
