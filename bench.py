@@ -49,12 +49,13 @@ FLUSH_BYTES = 256 << 20       # the flush writes a buffer twice the L2 size
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 _CSRC = "mla_decode_attention_etap_b200/csrc/"
-# The sources each decode kernel is built from (its ncu traffic figure is valid while they hash the same).
+# The sources each decode kernel is compiled from (its ncu traffic figure is valid while they hash the
+# same); the plan and combine kernels are separate kernels with their own sources.
 KERNEL_SOURCES = {
     "etap_pair_kernel": [_CSRC + f for f in ("etap_pair_kernel.cuh", "etap_common.cuh", "ptx_sm100.cuh",
                                              "plan_core.h", "merge.cuh")],
     "etap_duo_kernel": [_CSRC + f for f in ("etap_duo_kernel.cuh", "etap_common.cuh", "ptx_sm100.cuh",
-                                            "plan_core.h", "plan_combine_kernels.cuh", "merge.cuh")],
+                                            "plan_core.h")],
 }
 PROFILE_SUMMARIES = {
     "etap_pair_kernel": [os.path.join(ROOT, "profiles", "etap_pair_kernel_ncu.md"),

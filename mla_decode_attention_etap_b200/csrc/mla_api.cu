@@ -11,6 +11,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "mla_decode.h"
 #include "etap_pair_kernel.cuh"
@@ -18,6 +19,7 @@
 #include "plan_combine_kernels.cuh"
 #include "untransposed_kernel.cuh"
 #include "plan_core.h"
+#include "plan_cut.h"
 #include "form_ablation.cuh"
 #include "stream_probe.cuh"
 
@@ -249,33 +251,47 @@ int mla_decode_plan_host(const int32_t *seqlens, int batch, int q_len, int num_h
         unit_rows = mla::kDuoRows;
         gcols = mla::duo_group_cols(mode);
     }
-    int64_t total = 0;
-    for (int b = 0; b < batch; ++b) total += mla::units_of(seqlens[b], unit_rows);
+    // the cost-balanced cut of plan_core.h, sequence by sequence as the plan kernel does it
+    const int E = mla::end_cost_units(unit_rows);
+    int64_t total = 0, total_cost = 0;
+    for (int b = 0; b < batch; ++b) {
+        const int u = mla::units_of(seqlens[b], unit_rows);
+        total += u;
+        total_cost += u + (u > 0 ? E : 0);
+    }
     if (total > INT32_MAX) return MLA_ERR_UNSUPPORTED;
     const int used = mla::used_ctas(total, ctas);
-    if (cta_ranges)
-        for (int c = 0; c < ctas; ++c) {
-            cta_ranges[2 * c] = (int32_t)mla::cta_begin(total, used, c);
-            cta_ranges[2 * c + 1] = (int32_t)mla::cta_begin(total, used, c + 1);
-        }
-    if (seq_info) {
-        int64_t off = 0;
-        int slots = 0;
-        for (int b = 0; b < batch; ++b) {
-            const int64_t t0 = off, t1 = off + mla::units_of(seqlens[b], unit_rows);
-            int first = -1, nsplit = 0;
-            if (t1 > t0) {
-                first = mla::cta_of(total, used, t0);
-                nsplit = mla::cta_of(total, used, t1 - 1) - first + 1;
+    std::vector<int32_t> begin((size_t)ctas + 1, (int32_t)total);
+    int64_t f = 0, g = 0;
+    int slots = 0;
+    for (int b = 0; b < batch; ++b) {
+        const int64_t units = mla::units_of(seqlens[b], unit_rows);
+        const int64_t gend = g + units + (units > 0 ? E : 0);
+        int first = -1, nsplit = 0;
+        if (units > 0) {
+            first = mla::cta_of(total_cost, used, g);
+            nsplit = mla::cta_of(total_cost, used, g + units - 1) - first + 1;
+            for (int c = mla::first_range_at_or_after(total_cost, used, g); c < used; ++c) {
+                const int64_t x = mla::cta_begin(total_cost, used, c);
+                if (x >= gend) break;
+                begin[c] = (int32_t)mla::unit_at_cost(x, g, f, units);
             }
-            seq_info[4 * b + 0] = (int32_t)(t1 - t0);
+        }
+        if (seq_info) {
+            seq_info[4 * b + 0] = (int32_t)units;
             seq_info[4 * b + 1] = first;
             seq_info[4 * b + 2] = nsplit;
             seq_info[4 * b + 3] = slots;
-            if (nsplit >= 2) slots += nsplit;
-            off = t1;
         }
+        if (nsplit >= 2) slots += nsplit;
+        f += units;
+        g = gend;
     }
+    if (cta_ranges)
+        for (int c = 0; c < ctas; ++c) {
+            cta_ranges[2 * c] = begin[c];
+            cta_ranges[2 * c + 1] = begin[c + 1];
+        }
     if (num_ctas_out) *num_ctas_out = ctas;
     if (num_groups_out) *num_groups_out = groups;
     if (unit_rows_out) *unit_rows_out = unit_rows;

@@ -7,6 +7,7 @@
 #include "etap_common.cuh"
 #include "merge.cuh"
 #include "plan_core.h"
+#include "plan_cut.h"
 
 namespace mla {
 
@@ -52,9 +53,9 @@ __device__ __forceinline__ int block_min(int x, int *smem32) {
     return r;
 }
 
-// One schedule: unit prefix sums, per-CTA flattened ranges, per-sequence split info and
-// zeroed merge counters, plus its header words.  Every thread of the block calls it; thread i
-// owns the consecutive sequences [b0, b1).
+// One schedule: unit prefix sums, per-CTA flattened ranges (cut by cost, see plan_core.h),
+// per-sequence split info and zeroed merge counters, plus its header words.  Every thread of the
+// block calls it; thread i owns the consecutive sequences [b0, b1).
 __device__ void plan_schedule(const int32_t *__restrict__ seqlens, int batch, int b0, int b1, int ctas, int groups,
                               int unit_rows, int gcols, int mode, int32_t *__restrict__ ws, const Sched &sc, int hdr,
                               int64_t *scan_smem) {
@@ -63,43 +64,61 @@ __device__ void plan_schedule(const int32_t *__restrict__ seqlens, int batch, in
     int32_t *seq_info = ws + sc.seq_info / 4;
     int32_t *counters = ws + sc.counters / 4;
     int32_t *cta_seq = ws + sc.cta_seq / 4;
-    // flattened unit offsets: exclusive prefix sum of units per sequence
-    int64_t mine = 0;
-    for (int b = b0; b < b1; ++b) mine += units_of(seqlens[b], unit_rows);
-    int64_t total;
+    const int E = end_cost_units(unit_rows);
+    // flattened unit offsets and cost offsets: exclusive prefix sums per sequence
+    int64_t mine = 0, mine_cost = 0;
+    for (int b = b0; b < b1; ++b) {
+        const int u = units_of(seqlens[b], unit_rows);
+        mine += u;
+        mine_cost += u + (u > 0 ? E : 0);
+    }
+    int64_t total, total_cost;
     int64_t f = block_exclusive_scan(mine, scan_smem, &total);
+    int64_t g = block_exclusive_scan(mine_cost, scan_smem, &total_cost);
     const int used = used_ctas(total, ctas);
-    // splits per sequence (the consecutive CTAs its units fall on)
+    for (int c = threadIdx.x; c < ctas; c += blockDim.x) {
+        cta_seq[c] = batch;  // no units, unless a sequence below claims it
+        if (c >= used) ranges[2 * c] = (int32_t)total;
+    }
+    // range starts that fall inside each sequence's cost interval, and its split CTAs
     int64_t split_slots = 0;
     for (int b = b0; b < b1; ++b) {
-        const int64_t t0 = f, t1 = f + units_of(seqlens[b], unit_rows);
+        const int64_t units = units_of(seqlens[b], unit_rows);
+        const int64_t t0 = f, t1 = f + units;
+        const int64_t gend = g + units + (units > 0 ? E : 0);
         int first = -1, nsplit = 0;
-        if (t1 > t0) {
-            first = cta_of(total, used, t0);
-            nsplit = cta_of(total, used, t1 - 1) - first + 1;
+        if (units > 0) {
+            first = cta_of(total_cost, used, g);
+            nsplit = cta_of(total_cost, used, g + units - 1) - first + 1;
+            for (int c = first_range_at_or_after(total_cost, used, g); c < used; ++c) {
+                const int64_t x = cta_begin(total_cost, used, c);
+                if (x >= gend) break;
+                ranges[2 * c] = (int32_t)unit_at_cost(x, g, t0, units);
+            }
         }
         tile_off[b] = (int32_t)t0;
-        // the units whose range starts inside this sequence start their walk here
-        for (int c = first; c >= 0 && c < first + nsplit; ++c)
-            if (cta_begin(total, used, c) >= t0) cta_seq[c] = b;
-        seq_info[4 * b + 0] = (int32_t)(t1 - t0);
+        seq_info[4 * b + 0] = (int32_t)units;
         seq_info[4 * b + 1] = first;
         seq_info[4 * b + 2] = nsplit;
         if (nsplit >= 2) split_slots += nsplit;
         f = t1;
+        g = gend;
     }
-    // partial-output slots: exclusive prefix sum of the split counts of split sequences
+    // partial-output slots: exclusive prefix sum of the split counts of split sequences (the scan's
+    // barriers also publish every range start written above)
     int64_t slots;
     int64_t sl = block_exclusive_scan(split_slots, scan_smem, &slots);
     for (int b = b0; b < b1; ++b) {
         seq_info[4 * b + 3] = (int32_t)sl;
-        if (seq_info[4 * b + 2] >= 2) sl += seq_info[4 * b + 2];
+        const int nsplit = seq_info[4 * b + 2];
+        if (nsplit >= 2) sl += nsplit;
+        // the units whose range starts inside this sequence start their walk here
+        const int first = seq_info[4 * b + 1];
+        for (int c = first; c >= 0 && c < first + nsplit; ++c)
+            if (ranges[2 * c] >= tile_off[b]) cta_seq[c] = b;
     }
-    for (int c = threadIdx.x; c < ctas; c += blockDim.x) {
-        ranges[2 * c] = (int32_t)cta_begin(total, used, c);
-        ranges[2 * c + 1] = (int32_t)cta_begin(total, used, c + 1);
-        if (c >= used) cta_seq[c] = batch;  // no units
-    }
+    for (int c = threadIdx.x; c < ctas; c += blockDim.x)
+        ranges[2 * c + 1] = c + 1 < ctas ? ranges[2 * (c + 1)] : (int32_t)total;
     for (int i = threadIdx.x; i < 2 * batch * groups; i += blockDim.x) counters[i] = 0;
     for (int i = threadIdx.x; i < batch; i += blockDim.x) ws[sc.done / 4 + i] = 0;
     if (threadIdx.x == 0) {

@@ -1,10 +1,10 @@
 // Split-KV schedules and workspace layout, shared by the device plan kernel,
 // the decode/combine kernels and the host mirror (mla_decode_plan_host).
 //
-// The KV units of all sequences are concatenated in sequence order; unit range
-// c of a column group takes the flattened units [T*c/G, T*(c+1)/G).  A sequence
-// touched by several ranges is "split": each writes an fp32 partial (O_s, lse_s)
-// into its slot and the merge (in the decode kernel, or the combine kernel)
+// The KV units of all sequences are concatenated in sequence order and cut into one
+// contiguous range per work unit and column group, balanced by cost (plan_cut.h).  A
+// sequence touched by several ranges is "split": each writes an fp32 partial (O_s,
+// lse_s) into its slot and the merge (in the decode kernel, or the combine kernel)
 // combines them.  Not on the pages: it exists so that a batch of few long
 // sequences still spreads over every SM.
 //
@@ -71,15 +71,14 @@ MLA_HD int tiles_of(int L) { return units_of(L, kTileRows); }
 // The duo mode the plan picks for these lengths (min_len: shortest nonempty sequence, 0 if none).
 MLA_HD int duo_mode(int ncols, int min_len) { return duo_mode1_possible(ncols) && min_len >= kSingleP_MinRows ? 1 : 0; }
 
-// CTAs that receive work: never more than there are units, so that every CTA
-// in [0, used) owns at least one unit and the idle ones all come last (a
-// sequence's splits are then exactly the consecutive CTAs that touch it).
+// Work units that receive ranges: never more than there are units.
 MLA_HD int used_ctas(int64_t total, int ctas) { return total < (int64_t)ctas ? (int)total : ctas; }
-// First flattened unit of CTA c: CTA c covers [cta_begin(c), cta_begin(c+1)).
+// Near-equal cut of [0, total) into `used` ranges: range c is [cta_begin(c), cta_begin(c+1)).
+// The plan cuts the cost axis of plan_cut.h this way.
 MLA_HD int64_t cta_begin(int64_t total, int used, int c) {
     return c >= used ? total : total * (int64_t)c / used;
 }
-// The CTA whose range holds flattened unit f (0 <= f < total, used >= 1).
+// The range that holds position f (0 <= f < total, used >= 1).
 MLA_HD int cta_of(int64_t total, int used, int64_t f) { return (int)(((f + 1) * (int64_t)used - 1) / total); }
 
 MLA_HD size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }

@@ -16,6 +16,35 @@ def units(L, rows):
     return 0 if L <= 0 else (L + rows - 1) // rows
 
 
+def end_cost(rows):
+    """Units a sequence end counts for when the ranges are cut (plan_core.h: end_cost_units)."""
+    return 4 if rows == 128 else 2
+
+
+def cost_cut(lens, rows, ctas):
+    """The cost-balanced cut written out directly: the cost axis holds each nonempty sequence's units
+    followed by end_cost(rows) end positions; it is cut into min(T, ctas) near-equal pieces, and each
+    cut lands on the unit it falls on (or, among a sequence's end positions, on its last boundary)."""
+    us = [units(int(L), rows) for L in lens]
+    T = sum(us)
+    used = min(T, ctas)
+    C = sum(u + (end_cost(rows) if u else 0) for u in us)
+    begins = []
+    for c in range(ctas):
+        if c >= used:
+            begins.append(T)
+            continue
+        x = C * c // used
+        g = f = 0
+        for u in us:
+            gend = g + u + (end_cost(rows) if u else 0)
+            if u and g <= x < gend:
+                begins.append(f + min(x - g, u))
+                break
+            g, f = gend, f + u
+    return [(begins[c], begins[c + 1] if c + 1 < ctas else T) for c in range(ctas)]
+
+
 def expected_grouping(lens, q, h, n_sms, schedule):
     """(unit_rows, group_cols, groups, ctas) as the pages' decode path is laid out here."""
     ncols = q * h
@@ -45,15 +74,26 @@ def test_schedule_invariants(seed, schedule, n_sms, h, q):
     ranges, info, ctas, groups, rows, gcols = m.mla_decode_plan_host(lens, q, h, n_sms, schedule)
     assert (rows, gcols, groups, ctas) == expected_grouping(lens, q, h, n_sms, schedule)
     T = sum(units(int(L), rows) for L in lens)
-    # the unit ranges tile [0, T) in order; the working units come first, each with at least one
-    # unit of KV, sizes within 1 of each other; idle ones (only when T < ctas) come last
+    # the unit ranges tile [0, T) in order, cut by cost (each sequence end counts as extra units)
     assert ranges[0, 0] == 0 and ranges[-1, 1] == T
     assert np.all(ranges[1:, 0] == ranges[:-1, 1])
+    assert [tuple(r) for r in ranges.tolist()] == cost_cut(lens, rows, ctas)
     sizes = ranges[:, 1] - ranges[:, 0]
     used = min(ctas, T)
-    assert np.all(sizes[:used] >= 1) and np.all(sizes[used:] == 0)
+    assert np.all(sizes[used:] == 0)
     if used:
-        assert sizes[:used].max() - sizes[:used].min() <= 1
+        # a range's units plus the end costs it carries stay within one end cost + 1 of the fair share
+        ends = np.zeros(ctas, np.int64)
+        off = 0
+        for L in lens:
+            u = units(int(L), rows)
+            if u:
+                last = off + u - 1
+                ends[int(np.searchsorted(ranges[:, 1], last, side="right"))] += 1
+            off += u
+        cost = sizes + end_cost(rows) * ends
+        C = T + end_cost(rows) * int(sum(1 for L in lens if units(int(L), rows)))
+        assert np.all(np.abs(cost[:used] - C / used) <= end_cost(rows) + 1)
     # per sequence: the units that own some of its rows are exactly [first, first + nsplit)
     off = 0
     slots = 0
@@ -89,11 +129,15 @@ def test_fewer_units_than_ctas(lens, n_sms, h):
 
 
 def test_headline_shape_balance():
+    """16 x 512 tiles over 74 CTA pairs: a pair that holds a sequence end takes about 4 tiles fewer."""
     ranges, info, ctas, groups, rows, gcols = m.mla_decode_plan_host([65536] * 16, 1, 16, 148)
     assert (ctas, groups, rows, gcols) == (74, 1, 128, 16)
     sizes = ranges[:, 1] - ranges[:, 0]
-    assert sizes.min() == 110 and sizes.max() == 111
-    assert np.all(info[:, 2] >= 5)
+    assert sizes.sum() == 8192 and sizes.min() >= 107 and sizes.max() <= 112
+    ends = [int(np.searchsorted(ranges[:, 1], 512 * (b + 1) - 1, side="right")) for b in range(16)]
+    others = np.setdiff1d(np.arange(74), ends)
+    assert sizes[ends].mean() + 3 < sizes[others].mean()
+    assert np.all(info[:, 2] >= 4)
 
 
 def test_h128_groups_depend_on_the_shortest_sequence():
