@@ -100,9 +100,6 @@ int ensure_smem_attr() {
         e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)mla::PairCfg16::SMEM_ALLOC);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-        e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)mla::PairCfg32::SMEM_ALLOC);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg16E4>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::PairCfg16E4::SMEM_ALLOC);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -117,9 +114,6 @@ int ensure_smem_attr() {
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg16, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::PairCfg16::SMEM_ALLOC);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-        e = cudaFuncSetAttribute(mla::etap_pair_kernel<mla::PairCfg32, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::PairCfg32::SMEM_ALLOC);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         e = cudaFuncSetAttribute(mla::untransposed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)mla::kUtSmemAlloc);
@@ -441,9 +435,10 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
     p.slots = lay.slots;
     p.trace = trace;
     p.trace_cap = trace ? trace_cap : 0;
-    // splits of a sequence are at most the work units (CTA pairs per column group)
+    // splits of a sequence are at most the work units (CTA pairs per column group); the bf16 cache
+    // reaches the pair kernel only with 16 columns (more run the M = 256 kernel)
     const int max_splits = fp8 ? (ng == 16 ? mla::PairCfg16E4::MERGE_MAX_SPLITS : mla::PairCfg32E4::MERGE_MAX_SPLITS)
-                               : (ng == 16 ? mla::PairCfg16::MERGE_MAX_SPLITS : mla::PairCfg32::MERGE_MAX_SPLITS);
+                               : mla::PairCfg16::MERGE_MAX_SPLITS;
     const bool separate_combine = !(flags & MLA_FLAG_SKIP_COMBINE) && lay.ctas > max_splits;
     p.fuse_merge = ((flags & MLA_FLAG_SKIP_COMBINE) || separate_combine) ? 0 : 1;
 
@@ -522,8 +517,7 @@ int decode_fwd_impl(const void *q, const void *kv, const float *kv_scale, const 
         e = ng == 16 ? launch_pair<mla::PairCfg16E4>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s)
                      : launch_pair<mla::PairCfg32E4>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s);
     else
-        e = ng == 16 ? launch_pair<mla::PairCfg16>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s)
-                     : launch_pair<mla::PairCfg32>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s);
+        e = launch_pair<mla::PairCfg16>(tm_q, tm_kv, tm_qr, tm_kvr, p, clusters, s);
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "etap_pair_kernel launch");
