@@ -89,11 +89,13 @@ MLA_API size_t mla_decode_workspace_size(int batch, int q_len, int num_heads, in
 /*
  * Split-KV scheduling metadata (not on the pages: needed so that a batch with
  * few sequences still fills every SM). Reads seqlens (device int32[batch]),
- * cuts the concatenated KV tiles (128 rows each) of all sequences into
- * num_ctas near-equal contiguous ranges, and records for each sequence how
- * many ranges touch it and where its partial results go. One small kernel;
- * no host synchronisation, so the call can be captured in a CUDA graph.
- * Also clears the workspace status word.
+ * concatenates the KV units of all sequences (128 rows each for the CTA-pair
+ * kernel, 256 for the M = 256 kernel), cuts them into one contiguous range per
+ * work unit and column group, balanced by cost (each sequence end counts as the
+ * units its epilogue and merge take, so a range may be empty), and records for
+ * each sequence how many ranges touch it and where its partial results go. One
+ * small kernel; no host synchronisation, so the call can be captured in a CUDA
+ * graph. Also clears the workspace status word.
  */
 MLA_API int mla_decode_plan(const int32_t *seqlens, int batch, int q_len, int num_heads, int num_sms,
                     void *workspace, size_t workspace_bytes, void *stream);
@@ -274,7 +276,8 @@ MLA_API int mla_decode_read_status(const void *workspace, int *status_out, void 
  * a pair) and column groups of 64, or of 128 when q_len*h > 64 and every nonempty sequence
  * holds at least 8192 rows (the plan picks this on the device from the same lengths); for
  * q_len*h <= 16 it is schedule 0. Writes, when the pointers are non-NULL:
- *   cta_ranges  int32[num_ctas*2]  flattened unit range [begin, end) of each work unit
+ *   cta_ranges  int32[num_ctas*2]  flattened unit range [begin, end) of each work unit (cut by
+ *                                  cost as mla_decode_plan does; possibly empty)
  *   seq_info    int32[batch*4]     per sequence: unit count, first work unit, number of splits, partial slot offset
  * and returns the work units per column group, the column groups, the rows per unit and the
  * columns per group through the output pointers (each may be NULL).
