@@ -2,7 +2,9 @@
 """Benchmark of MLA decode attention (ETAP form) on B200.
 
 One step = one pass of the whole decode path over one batch: split-KV plan,
-ETAP decode kernel (which also merges the split-KV partials, log-sum-exp).  Default workload: B=16 sequences,
+ETAP decode kernel, and the log-sum-exp merge of the split-KV partials (inside
+the CTA-pair kernel; a combine kernel behind the M = 256 kernel that serves the
+bf16 cache above 16 query columns).  Default workload: B=16 sequences,
 16 heads, one query token, 65536 contiguous cache rows each (1.21 GB of bf16
 latent KV, larger than the 126 MB L2, so no flush is needed between steps;
 workloads smaller than L2 get a 256 MB write before every timed step, outside
@@ -19,6 +21,7 @@ fp64 oracle timed on the host as a CPU baseline, and GPU clocks sampled while th
 steps run.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+  python bench.py --workload NAME --form untransposed   # the same decode in the S = Q K^T form
   python bench.py --ablation    # transposed vs untransposed tensor-core cost per KV tile
 
 N > 1 runs under torchrun, one process per GPU; every rank decodes its own
